@@ -1,0 +1,319 @@
+"""Block-scaled int8 projection for NVIDIA B200 (sm_100a).
+
+Thin ctypes binding over the C ABI of ``libbsr.so`` (declared in
+``include/bsr.h``).  The functions here only marshal arguments: they check
+dtypes, shapes and devices of ``torch.Tensor`` arguments, take raw device
+pointers and the current CUDA stream, and call the library; every step of the
+computation runs in the library's CUDA kernels.  PyTorch is used for device
+memory and streams only.  There is no CPU fallback: if the library cannot be
+loaded, every call raises.
+
+Operations (gemm_dense_int8.rs launcher page):
+
+* :func:`requant_w` -- ``requant_w_nvfp4_int8``: NVFP4 weight -> int8 codes +
+  one F32 scale per 32 elements (scale2 folded in).
+* :func:`requant_a` -- ``requant_a_kernel``: BF16 activations -> int8 codes +
+  block-major F32 scales.
+* :func:`gemm` -- ``faith2_kernel``: tcgen05 int8 GEMM with per-32-block
+  rescale, F32 accumulation, BF16 output.
+* :func:`proj` -- ``int8_gemm_faith2_prefill``: the whole projection from BF16
+  activations (decode kernel for M <= 16, requant_a + gemm otherwise).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "BsrError",
+    "lib",
+    "abi_version",
+    "last_error",
+    "device_status",
+    "requant_w",
+    "a_scale_ld",
+    "requant_a",
+    "gemm",
+    "gemm_partials",
+    "proj_scratch_bytes",
+    "proj",
+    "decode",
+    "DECODE_MAX_M",
+    "STATUS_NAMES",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libbsr.so")
+DECODE_MAX_M = 16
+
+STATUS_NAMES = {
+    0: "BSR_OK",
+    1: "BSR_EINVAL",
+    2: "BSR_EALIGN",
+    3: "BSR_ESHAPE",
+    4: "BSR_ESCRATCH",
+    5: "BSR_ECUDA",
+    6: "BSR_ETIMEOUT",
+    7: "BSR_ENODEV",
+}
+
+# (name, restype, argtypes) of every exported symbol, mirroring include/bsr.h
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+SIGNATURES = [
+    ("bsr_abi_version", ctypes.c_int, []),
+    ("bsr_last_error", ctypes.c_char_p, []),
+    ("bsr_device_status", ctypes.c_int, []),
+    ("bsr_requant_w", ctypes.c_int, [_P, _P, ctypes.c_float, _P, _P, _I64, _I64, _P]),
+    ("bsr_a_scale_ld", _I64, [_I64]),
+    ("bsr_requant_a", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
+    ("bsr_gemm", ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("bsr_proj_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
+    ("bsr_proj", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P]),
+    ("bsr_decode", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("bsr_gemm_partials", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+]
+
+
+class BsrError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        self.name = STATUS_NAMES.get(status, str(status))
+        super().__init__(f"{self.name}: {message}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbsr.so (built in-tree by ``build.py``); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m block_scaled_precision_requant_b200.build`"
+            )
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise BsrError(status, lib().bsr_last_error().decode())
+
+
+def abi_version() -> int:
+    return lib().bsr_abi_version()
+
+
+def last_error() -> str:
+    return lib().bsr_last_error().decode()
+
+
+def device_status() -> int:
+    """Synchronise and return/clear the device status word (0 = no wait timed out)."""
+    return lib().bsr_device_status()
+
+
+# ---------------------------------------------------------------------------
+# tensor marshalling helpers
+# ---------------------------------------------------------------------------
+
+
+def _torch():
+    import torch
+
+    return torch
+
+
+def _stream_ptr(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, dtype, shape, name):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _empty(shape, dtype, like):
+    torch = _torch()
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+# ---------------------------------------------------------------------------
+# operations
+# ---------------------------------------------------------------------------
+
+
+def requant_w(w_packed, w_e4m3, scale2: float, w_i8=None, w_scale=None, stream=None):
+    """NVFP4 weight -> (w_i8 [N, K] int8, w_scale [N, K/32] float32)."""
+    torch = _torch()
+    n, k2 = w_packed.shape
+    k = 2 * k2
+    if w_i8 is None:
+        w_i8 = _empty((n, k), torch.int8, w_packed)
+    if w_scale is None:
+        w_scale = _empty((n, k // 32), torch.float32, w_packed)
+    _check(
+        lib().bsr_requant_w(
+            _dev(w_packed, torch.uint8, (n, k2), "w_packed"),
+            _dev(w_e4m3, torch.uint8, (n, k // 16), "w_e4m3"),
+            ctypes.c_float(float(scale2)),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            n,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return w_i8, w_scale
+
+
+def a_scale_ld(m: int) -> int:
+    return lib().bsr_a_scale_ld(m)
+
+
+def requant_a(a, a_i8=None, a_scale_t=None, stream=None):
+    """BF16 [M, K] -> (a_i8 [M, K] int8, a_scale_t [K/32, ld] float32 block-major)."""
+    torch = _torch()
+    m, k = a.shape
+    ld = a_scale_ld(m)
+    if a_i8 is None:
+        a_i8 = _empty((m, k), torch.int8, a)
+    if a_scale_t is None:
+        a_scale_t = _empty((k // 32, ld), torch.float32, a)
+    _check(
+        lib().bsr_requant_a(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(a_i8, torch.int8, (m, k), "a_i8"),
+            _dev(a_scale_t, torch.float32, (k // 32, ld), "a_scale_t"),
+            m,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return a_i8, a_scale_t
+
+
+def gemm(a_i8, a_scale_t, w_i8, w_scale, out=None, stream=None):
+    """int8 block-scaled GEMM -> out [M, N] bfloat16."""
+    torch = _torch()
+    m, k = a_i8.shape
+    n = w_i8.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a_i8)
+    _check(
+        lib().bsr_gemm(
+            _dev(a_i8, torch.int8, (m, k), "a_i8"),
+            _dev(a_scale_t, torch.float32, (k // 32, a_scale_ld(m)), "a_scale_t"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def gemm_partials(a_i8, a_scale_t, w_i8, w_scale, out=None, partials=None, stream=None):
+    """:func:`gemm` that also returns the int32 block partials [M, N, K/32]."""
+    torch = _torch()
+    m, k = a_i8.shape
+    n = w_i8.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a_i8)
+    if partials is None:
+        partials = _empty((m, n, k // 32), torch.int32, a_i8)
+    _check(
+        lib().bsr_gemm_partials(
+            _dev(a_i8, torch.int8, (m, k), "a_i8"),
+            _dev(a_scale_t, torch.float32, (k // 32, a_scale_ld(m)), "a_scale_t"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            _dev(partials, torch.int32, (m, n, k // 32), "partials"),
+            m,
+            n,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return out, partials
+
+
+def proj_scratch_bytes(m: int, k: int) -> int:
+    return lib().bsr_proj_scratch_bytes(m, k)
+
+
+def proj(a, w_i8, w_scale, out=None, scratch=None, stream=None):
+    """out [M, N] bfloat16 = A [M, K] (bfloat16) . W^T from the requantised weight."""
+    torch = _torch()
+    m, k = a.shape
+    n = w_i8.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    need = proj_scratch_bytes(m, k)
+    if scratch is None and need:
+        scratch = _empty((need,), torch.uint8, a)
+    sp = ctypes.c_void_p(scratch.data_ptr()) if scratch is not None else ctypes.c_void_p(0)
+    sb = scratch.numel() * scratch.element_size() if scratch is not None else 0
+    if scratch is not None and not scratch.is_cuda:
+        raise ValueError("scratch must be a CUDA tensor")
+    _check(
+        lib().bsr_proj(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            sp,
+            sb,
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def decode(a, w_i8, w_scale, out=None, stream=None):
+    """The decode kernel for any M (activation requantisation fused, CUDA cores)."""
+    torch = _torch()
+    m, k = a.shape
+    n = w_i8.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    _check(
+        lib().bsr_decode(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return out

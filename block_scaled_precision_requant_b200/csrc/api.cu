@@ -1,0 +1,264 @@
+// C ABI of libbsr.so: argument validation, tensor-map encoding, launches.
+// Declarations and the contract of every entry point are in include/bsr.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "bsr.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+// Device status word (one per device that loads the library); kernels get
+// its address as an argument.
+__device__ int g_dev_status = 0;
+
+thread_local char g_err[512] = {0};
+
+bsr_status fail(bsr_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bsr_status ok() {
+  g_err[0] = 0;
+  return BSR_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device properties, queried once per device.
+struct DevInfo {
+  int num_sms = 0;
+  size_t smem_optin = 0;
+  int cc_major = 0;
+  int* status = nullptr;  // device address of g_dev_status
+};
+
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+bsr_status device_info(DevInfo& out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(BSR_ENODEV, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(BSR_ENODEV, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (d.num_sms == 0) {
+    int sms = 0, smem = 0, major = 0;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+      return fail(BSR_ENODEV, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+    void* st = nullptr;
+    if ((e = cudaGetSymbolAddress(&st, g_dev_status)) != cudaSuccess)
+      return fail(BSR_ENODEV, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+    d.num_sms = sms;
+    d.smem_optin = (size_t)smem;
+    d.cc_major = major;
+    d.status = static_cast<int*>(st);
+  }
+  if (d.cc_major != 10) return fail(BSR_ENODEV, "device %d has compute capability %d.x, need 10.x (sm_100a)", dev, d.cc_major);
+  out = d;
+  return BSR_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bsr_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw,
+                     const char* what) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(BSR_ECUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {pitch_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSR_ECUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
+  return BSR_OK;
+}
+
+bsr_status check_dims(int64_t m, int64_t n, int64_t k, bool need_m, bool need_n) {
+  if ((need_m && (m < 0 || m > BSR_MAX_DIM)) || (need_n && (n < 0 || n > BSR_MAX_DIM)) || k < 0 ||
+      k > BSR_MAX_DIM)
+    return fail(BSR_EINVAL, "dimension out of range (m=%lld n=%lld k=%lld)", (long long)m, (long long)n,
+                (long long)k);
+  if (k == 0 || k % 32 != 0) return fail(BSR_ESHAPE, "K=%lld must be a positive multiple of 32", (long long)k);
+  return BSR_OK;
+}
+
+bsr_status cuda_status(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(BSR_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int64_t a_scale_ld(int64_t m) { return (m + 3) / 4 * 4; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
+                     uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (k % 128 != 0) return fail(BSR_ESHAPE, "bsr_gemm needs K %% 128 == 0 (K=%lld)", (long long)k);
+  if (m == 0 || n == 0) return ok();
+  if (!a_i8 || !a_scale_t || !w_i8 || !w_scale || !out) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(a_i8) || !aligned16(a_scale_t) || !aligned16(w_i8) || !aligned16(w_scale) ||
+      (reinterpret_cast<uintptr_t>(out) & 1u))
+    return fail(BSR_EALIGN, "bsr_gemm: pointers must be 16-byte aligned (out: 2-byte)");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  if (bsr::gemm_smem_bytes() > d.smem_optin)
+    return fail(BSR_ENODEV, "device shared memory %zu < %zu", d.smem_optin, bsr::gemm_smem_bytes());
+  bsr::GemmMaps maps;
+  const int64_t nb = k / 32;
+  if ((st = encode_2d(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_i8, k, n, k, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B, "w_i8")) != BSR_OK ||
+      (st = encode_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_i8, k, m, k, 128, 128,
+                      CU_TENSOR_MAP_SWIZZLE_128B, "a_i8")) != BSR_OK ||
+      (st = encode_2d(&maps.ws, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w_scale, nb, n, nb * 4, 4, 128,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, "w_scale")) != BSR_OK ||
+      (st = encode_2d(&maps.as, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a_scale_t, m, nb, a_scale_ld(m) * 4, 128, 4,
+                      CU_TENSOR_MAP_SWIZZLE_NONE, "a_scale_t")) != BSR_OK)
+    return st;
+  return cuda_status(bsr::launch_gemm(maps, out, partials, d.status, (int)m, (int)n, (int)k, as_stream(stream), d.num_sms),
+                     "gemm launch");
+}
+
+bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                       int64_t n, int64_t k, void* stream) {
+  DevInfo d;
+  bsr_status st;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  const int mr = bsr::decode_rows_per_cta((int)m, (int)k, d.smem_optin);
+  if (mr == 0) return fail(BSR_ESHAPE, "K=%lld too large for the decode kernel's shared memory", (long long)k);
+  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, as_stream(stream),
+                                        d.num_sms),
+                     "decode launch");
+}
+
+bsr_status check_proj_args(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out) {
+  if (!a || !w_i8 || !w_scale || !out) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(a) || !aligned16(w_i8) || !aligned16(w_scale) || (reinterpret_cast<uintptr_t>(out) & 1u))
+    return fail(BSR_EALIGN, "a, w_i8, w_scale must be 16-byte aligned, out 2-byte aligned");
+  return BSR_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsr_abi_version(void) { return BSR_ABI_VERSION; }
+
+const char* bsr_last_error(void) { return g_err; }
+
+int bsr_device_status(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(int)) != cudaSuccess) return -1;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+  return v;
+}
+
+bsr_status bsr_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2, int8_t* w_i8,
+                         float* w_scale, int64_t n, int64_t k, void* stream) {
+  bsr_status st = check_dims(0, n, k, false, true);
+  if (st != BSR_OK) return st;
+  if (n == 0) return ok();
+  if (!w_packed || !w_e4m3 || !w_i8 || !w_scale) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(w_packed) || !aligned16(w_e4m3) || !aligned16(w_i8) || !aligned16(w_scale))
+    return fail(BSR_EALIGN, "bsr_requant_w: pointers must be 16-byte aligned");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  return cuda_status(bsr::launch_requant_w(w_packed, w_e4m3, scale2, w_i8, w_scale, n, k, as_stream(stream),
+                                           d.num_sms),
+                     "requant_w launch");
+}
+
+int64_t bsr_a_scale_ld(int64_t m) { return m < 0 ? 0 : a_scale_ld(m); }
+
+bsr_status bsr_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, int64_t m, int64_t k, void* stream) {
+  bsr_status st = check_dims(m, 0, k, true, false);
+  if (st != BSR_OK) return st;
+  if (m == 0) return ok();
+  if (!a || !a_i8 || !a_scale_t) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(a) || !aligned16(a_i8) || !aligned16(a_scale_t))
+    return fail(BSR_EALIGN, "bsr_requant_a: pointers must be 16-byte aligned");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  return cuda_status(bsr::launch_requant_a(a, a_i8, a_scale_t, (int)m, (int)k, (int)a_scale_ld(m),
+                                           as_stream(stream), d.num_sms),
+                     "requant_a launch");
+}
+
+bsr_status bsr_gemm(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
+                    uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream) {
+  return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
+}
+
+bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
+                             uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream) {
+  if (!partials) return fail(BSR_EINVAL, "null partials");
+  return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, partials, m, n, k, stream);
+}
+
+size_t bsr_proj_scratch_bytes(int64_t m, int64_t k) {
+  if (m <= BSR_DECODE_MAX_M || k <= 0 || k % 128 != 0) return 0;
+  return align256((size_t)m * (size_t)k) + (size_t)(k / 32) * (size_t)a_scale_ld(m) * 4;
+}
+
+bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                      int64_t n, int64_t k, void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if ((st = check_proj_args(a, w_i8, w_scale, out)) != BSR_OK) return st;
+  return decode_impl(a, w_i8, w_scale, out, m, n, k, stream);
+}
+
+bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m, int64_t n,
+                    int64_t k, void* scratch, size_t scratch_bytes, void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if ((st = check_proj_args(a, w_i8, w_scale, out)) != BSR_OK) return st;
+  if (m <= BSR_DECODE_MAX_M || k % 128 != 0) return decode_impl(a, w_i8, w_scale, out, m, n, k, stream);
+  const size_t need = bsr_proj_scratch_bytes(m, k);
+  if (!scratch || scratch_bytes < need)
+    return fail(BSR_ESCRATCH, "scratch of %zu bytes needed, %zu given", need, scratch ? scratch_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
+  int8_t* a_i8 = static_cast<int8_t*>(scratch);
+  float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
+  if ((st = bsr_requant_a(a, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
+  return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,29 @@
+// Internal launch interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace bsr {
+
+struct GemmMaps {
+  CUtensorMap w;   // W_i8 [N, K] int8, box 128 x 128 B, 128-byte swizzle
+  CUtensorMap a;   // a_i8 [M, K] int8, box 128 x 128 B, 128-byte swizzle
+  CUtensorMap ws;  // W_scale [N, K/32] f32, box 128 x 4
+  CUtensorMap as;  // a_scale_t [K/32, ld] f32 (dims K/32 x M), box 4 x 128
+};
+
+cudaError_t launch_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2, int8_t* w_i8,
+                             float* w_scale, long long n, long long k, cudaStream_t stream, int num_sms);
+cudaError_t launch_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, int m, int k, int ld,
+                             cudaStream_t stream, int num_sms);
+int decode_rows_per_cta(int m, int k, size_t smem_limit);
+cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
+                          int k, int mr, cudaStream_t stream, int num_sms);
+size_t gemm_smem_bytes();
+cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
+                        cudaStream_t stream, int num_sms);
+
+}  // namespace bsr

@@ -1,0 +1,222 @@
+// Requantisation kernels (HBM-bound):
+//
+//  * requant_w: NVFP4 weight -> int8 codes + one F32 scale per 32 elements
+//    (gemm_dense_int8.rs, `requant_w_nvfp4_int8`: reads W_packed[N, K/2] and
+//    W_e4m3[N, K/16], folds the per-tensor scale2, writes W_i8[N, K] and
+//    W_scale[N, K/32]).
+//  * requant_a: BF16 activations -> int8 codes + one F32 scale per 32
+//    elements (gemm_dense_int8.rs, `requant_a_kernel` inside
+//    `int8_gemm_faith2_prefill`).  The scales are written block-major,
+//    a_scale_t[K/32][ld], which is the layout the tensor-core GEMM stages.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "quant.cuh"
+
+namespace bsr {
+
+// ---------------------------------------------------------------------------
+// requant_w
+//
+// One thread per 32-group: 16 packed bytes (32 E2M1 nibbles, element 2i in
+// the low nibble of byte i), two E4M3 block scales, 32 output codes and one
+// scale.  A 16-element block shares one E4M3 scale, so its dequantised values
+// take at most 8 magnitudes: v_i = RN((e2m1_i * e4m3) * scale2), i = 0..7.
+// The kernel quantises those 8 candidates once per block and maps every
+// nibble to its code with byte permutes; codes of negative nibbles are the
+// negated codes (rint half-even and the division are odd functions).
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
+  // hardware conversion E4M3 -> f16 (exact), then f16 -> f32 (exact)
+  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// E2M1 magnitude of index i (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_mag(uint32_t i) {
+  if (i == 0) return 0.0f;
+  if (i == 1) return 0.5f;
+  return __uint_as_float((((i >> 1) + 126u) << 23) | ((i & 1u) << 22));
+}
+
+// Largest nibble magnitude index (0..7) among the 16 nibbles of (x, y).
+__device__ __forceinline__ uint32_t max_mag_index(uint32_t x, uint32_t y) {
+  const uint32_t gx = (x & 0x77777777u) | 0x88888888u;
+  const uint32_t gy = (y & 0x77777777u) | 0x88888888u;
+  // nibble n >= t  <=>  ((8 + n) - t) keeps bit 3; no borrow crosses nibbles
+  auto any_ge = [&](uint32_t t) {
+    const uint32_t rep = t * 0x11111111u;
+    return (((gx - rep) | (gy - rep)) & 0x88888888u) != 0u;
+  };
+  uint32_t lo = any_ge(4) ? 4u : 0u;
+  lo += any_ge(lo + 2) ? 2u : 0u;
+  lo += any_ge(lo + 1) ? 1u : 0u;
+  return lo;
+}
+
+struct CodeTable {
+  uint32_t pos_lo, pos_hi, neg_lo, neg_hi;  // codes of magnitude index 0..7 (bytes)
+};
+
+__device__ __forceinline__ CodeTable block_codes(float s_e4m3, float scale2, const GroupScale& g) {
+  int q[8];
+  q[0] = 0;
+#pragma unroll
+  for (int i = 1; i < 8; ++i) {
+    const float v = __fmul_rn(e2m1_mag(i) * s_e4m3, scale2);  // e2m1 * e4m3 is exact
+    q[i] = (g.scale == 0.0f) ? 0 : quant_code(v, g);
+  }
+  CodeTable t;
+  t.pos_lo = pack4_s8(q[0], q[1], q[2], q[3]);
+  t.pos_hi = pack4_s8(q[4], q[5], q[6], q[7]);
+  t.neg_lo = pack4_s8(-q[0], -q[1], -q[2], -q[3]);
+  t.neg_hi = pack4_s8(-q[4], -q[5], -q[6], -q[7]);
+  return t;
+}
+
+// Byte permute in the PTX default mode: a selector nibble with bit 3 set
+// replicates the sign (bit 7) of the selected byte into the whole byte.
+__device__ __forceinline__ uint32_t prmt_sign(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Codes of the 8 nibbles of w (elements 0..7 of the word) -> two words.
+__device__ __forceinline__ uint2 map_word(uint32_t w, const CodeTable& t) {
+  const uint32_t sel0 = w & 0x7777u;
+  const uint32_t sel1 = (w >> 16) & 0x7777u;
+  // sign bits: odd nibbles' signs are the byte MSBs of w, even nibbles' are
+  // the byte MSBs of w << 4; replicate them into byte masks
+  const uint32_t ws = w << 4;
+  const uint32_t m0 = prmt_sign(ws, w, 0xD9C8u);
+  const uint32_t m1 = prmt_sign(ws, w, 0xFBEAu);
+  const uint32_t p0 = __byte_perm(t.pos_lo, t.pos_hi, sel0);
+  const uint32_t n0 = __byte_perm(t.neg_lo, t.neg_hi, sel0);
+  const uint32_t p1 = __byte_perm(t.pos_lo, t.pos_hi, sel1);
+  const uint32_t n1 = __byte_perm(t.neg_lo, t.neg_hi, sel1);
+  return make_uint2((p0 & ~m0) | (n0 & m0), (p1 & ~m1) | (n1 & m1));
+}
+
+__global__ void __launch_bounds__(256) requant_w_kernel(const uint4* __restrict__ w_packed,
+                                                        const uint16_t* __restrict__ w_e4m3, float scale2,
+                                                        uint4* __restrict__ w_i8, float* __restrict__ w_scale,
+                                                        long long groups) {
+  for (long long gi = (long long)blockIdx.x * blockDim.x + threadIdx.x; gi < groups;
+       gi += (long long)gridDim.x * blockDim.x) {
+    const uint4 p = __ldg(w_packed + gi);
+    const uint32_t e = __ldg(w_e4m3 + gi);
+    const float s0 = e4m3_to_f32(e & 0xFFu);
+    const float s1 = e4m3_to_f32(e >> 8);
+    const uint32_t i0 = max_mag_index(p.x, p.y);
+    const uint32_t i1 = max_mag_index(p.z, p.w);
+    const float a0 = fabsf(__fmul_rn(e2m1_mag(i0) * s0, scale2));
+    const float a1 = fabsf(__fmul_rn(e2m1_mag(i1) * s1, scale2));
+    const GroupScale g = group_scale(fmaxf(a0, a1));
+    const CodeTable t0 = block_codes(s0, scale2, g);
+    const CodeTable t1 = block_codes(s1, scale2, g);
+    const uint2 c0 = map_word(p.x, t0), c1 = map_word(p.y, t0);
+    const uint2 c2 = map_word(p.z, t1), c3 = map_word(p.w, t1);
+    w_i8[2 * gi] = make_uint4(c0.x, c0.y, c1.x, c1.y);
+    w_i8[2 * gi + 1] = make_uint4(c2.x, c2.y, c3.x, c3.y);
+    w_scale[gi] = g.scale;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// requant_a
+//
+// Four lanes per 32-group (8 BF16 each, one 16-byte load), eight groups per
+// warp taken from eight consecutive rows at the same block b, so the loads
+// are 64-byte row segments, the codes 32-byte segments and the eight scales
+// one 32-byte segment of the block-major scale array.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&x)[8]) {
+  x[0] = __uint_as_float(v.x << 16);
+  x[1] = __uint_as_float(v.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(v.y << 16);
+  x[3] = __uint_as_float(v.y & 0xFFFF0000u);
+  x[4] = __uint_as_float(v.z << 16);
+  x[5] = __uint_as_float(v.z & 0xFFFF0000u);
+  x[6] = __uint_as_float(v.w << 16);
+  x[7] = __uint_as_float(v.w & 0xFFFF0000u);
+}
+
+// Quantise 8 consecutive values of a group whose 4 lanes are adjacent
+// (lane & ~3 .. lane | 3).  Returns the 8 codes packed, and the group scale.
+__device__ __forceinline__ uint2 quant8_quad(const float (&x)[8], float& scale_out) {
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  const GroupScale g = group_scale(amax);
+  scale_out = g.scale;
+  int q[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) q[i] = (g.scale == 0.0f) ? 0 : quant_code(x[i], g);
+  return make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
+}
+
+__global__ void __launch_bounds__(256) requant_a_kernel(const uint4* __restrict__ a, uint2* __restrict__ a_i8,
+                                                        float* __restrict__ a_scale_t, int m, int k, int ld) {
+  const int lane = threadIdx.x & 31;
+  const int nb = k >> 5;
+  const long long tasks = (long long)((m + 7) >> 3) * nb;
+  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int sub = lane & 3;
+  for (long long t = warp0; t < tasks; t += nwarps) {
+    const int r8 = (int)(t / nb);
+    const int b = (int)(t - (long long)r8 * nb);
+    const int row = r8 * 8 + (lane >> 2);
+    const bool valid = row < m;  // uniform per group of 4 lanes
+    const long long e = (long long)(valid ? row : 0) * k + (long long)b * 32 + sub * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (valid) v = __ldg(a + (e >> 3));
+    float x[8];
+    bf16x8_to_f32(v, x);
+    float s;
+    const uint2 c = quant8_quad(x, s);
+    if (valid) {
+      a_i8[e >> 3] = c;
+      if (sub == 0) a_scale_t[(long long)b * ld + row] = s;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+
+static int grid_for(long long work_items, int per_block, int max_blocks) {
+  long long g = (work_items + per_block - 1) / per_block;
+  if (g < 1) g = 1;
+  if (g > max_blocks) g = max_blocks;
+  return (int)g;
+}
+
+cudaError_t launch_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2, int8_t* w_i8,
+                             float* w_scale, long long n, long long k, cudaStream_t stream, int num_sms) {
+  const long long groups = n * (k / 32);
+  const int grid = grid_for(groups, 256, num_sms * 8);
+  requant_w_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(w_packed),
+                                             reinterpret_cast<const uint16_t*>(w_e4m3), scale2,
+                                             reinterpret_cast<uint4*>(w_i8), w_scale, groups);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, int m, int k, int ld,
+                             cudaStream_t stream, int num_sms) {
+  const long long tasks = (long long)((m + 7) / 8) * (k / 32);
+  const int grid = grid_for(tasks, 8, num_sms * 8);
+  requant_a_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(a), reinterpret_cast<uint2*>(a_i8),
+                                             a_scale_t, m, k, ld);
+  return cudaGetLastError();
+}
+
+}  // namespace bsr

@@ -1,0 +1,175 @@
+/*
+ * bsr.h -- C ABI of the block-scaled int8 projection library (libbsr.so) for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The library computes the quantised projection out[M, N] = A[M, K] . W[N, K]^T
+ * described by the launcher page gemm_dense_int8.rs of the metrale
+ * model-layers ops crate:
+ *
+ *   1. `requant_w_nvfp4_int8` (doc comment): an NVFP4 weight -- packed E2M1
+ *      nibbles W_packed[N, K/2], one E4M3 scale per 16 elements W_e4m3[N, K/16],
+ *      one per-tensor F32 scale2 -- is requantised once to signed int8
+ *      W_i8[N, K] with one F32 scale per 32 elements W_scale[N, K/32]; the
+ *      caller keeps the result and reuses it ("ensure_int8_weight").
+ *   2. `int8_gemm_faith2_prefill` (doc comment): the BF16 activations A[M, K]
+ *      are requantised the same way (`requant_a_kernel`), then
+ *      `faith2_kernel` forms each 32-wide block's int32 dot product, multiplies
+ *      it by a_scale * w_scale, accumulates in F32 and writes BF16 out[M, N].
+ *
+ * Conventions fixed by this library where the page is silent:
+ *   - E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}, bit 3 = sign; element 2i of
+ *     a row is the low nibble of byte i.  E4M3 as in the OCP FP8 spec; the NaN
+ *     codes 0x7F / 0xFF are outside the contract (results unspecified).
+ *   - Dequantised weight v = (e2m1 * e4m3) * scale2 in float32.
+ *   - Per 32-element group: scale = RN_f32(amax / 127),
+ *     code = clamp(rint_half_even(RN_f32(x / scale)), -127, 127); an all-zero
+ *     group (or one whose scale underflows to 0) has scale 0 and codes 0.
+ *     Codes and scales are bit-exact with the CPU oracle in oracle/.
+ *   - Per block b the GPU adds RN(float(P) * w_scale) * a_scale into a float32
+ *     accumulator with one rounding (FMA); the order of the blocks' additions
+ *     is the library's, so BF16 outputs agree with the oracle within
+ *     |err| <= 2^-7 |ref| + 1e-3 rms(ref), not bit for bit.  Within one path
+ *     a row's output bits do not depend on M, on the other rows, on N or on
+ *     which rows of a stacked weight are launched together.
+ *
+ * Memory: every pointer is a device pointer (except where noted) owned by the
+ * caller; the library never allocates device memory.  All arrays are dense
+ * row-major.  Every call is asynchronous on `stream` (a cudaStream_t, NULL =
+ * the legacy default stream) and returns before the kernels finish.
+ *
+ * Errors: arguments are checked before anything is launched; on a non-OK
+ * status nothing was launched and bsr_last_error() returns a message (thread
+ * local).  M == 0 or N == 0 is a no-op that returns BSR_OK.  A CUDA launch
+ * failure returns BSR_ECUDA.  Kernels never trap: a pipeline wait that runs
+ * out (1 s) makes the kernel return early and sets a bit that
+ * bsr_device_status() reports.
+ */
+#ifndef BSR_H_
+#define BSR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSR_ABI_VERSION 1
+
+typedef enum bsr_status {
+  BSR_OK = 0,
+  BSR_EINVAL = 1,   /* null pointer, negative or too large dimension */
+  BSR_EALIGN = 2,   /* a pointer is not 16-byte aligned */
+  BSR_ESHAPE = 3,   /* K not a positive multiple of 32 (or of 128 where stated) */
+  BSR_ESCRATCH = 4, /* scratch missing or smaller than bsr_proj_scratch_bytes() */
+  BSR_ECUDA = 5,    /* a CUDA runtime/driver call failed */
+  BSR_ETIMEOUT = 6, /* reported by bsr_device_status() */
+  BSR_ENODEV = 7    /* no CUDA device, or not an sm_100 device */
+} bsr_status;
+
+/* Largest M, N or K accepted (the TMA coordinates are 32-bit). */
+#define BSR_MAX_DIM 2147483647LL
+
+/* Rows of A at or below which bsr_proj takes the decode path. */
+#define BSR_DECODE_MAX_M 16
+
+int bsr_abi_version(void);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+const char* bsr_last_error(void);
+
+/* Synchronises the current device, returns and clears the device status
+ * word: 0 if no kernel aborted a wait since the last call, else a bit set
+ * (1 TMA producer, 2 MMA issuer, 4 epilogue, 8 scale preparation timed out).
+ * Returns -1 if the device could not be queried. */
+int bsr_device_status(void);
+
+/*
+ * bsr_requant_w -- gemm_dense_int8.rs, `requant_w_nvfp4_int8`.
+ *   w_packed  [N, K/2]  uint8, two E2M1 codes per byte, low nibble first
+ *   w_e4m3    [N, K/16] uint8, E4M3 scale of each 16-element block
+ *   scale2    per-tensor F32 scale (host value), folded into w_scale
+ *   w_i8      [N, K]    int8 out: codes
+ *   w_scale   [N, K/32] float out: scale of each 32-element group
+ * Requirements: K > 0, K % 32 == 0; all pointers 16-byte aligned.
+ * HBM-bound; call once per weight and keep (w_i8, w_scale).
+ */
+bsr_status bsr_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2, int8_t* w_i8,
+                         float* w_scale, int64_t n, int64_t k, void* stream);
+
+/* Leading dimension (in floats) of the block-major activation scales for M
+ * rows: M rounded up to a multiple of 4. */
+int64_t bsr_a_scale_ld(int64_t m);
+
+/*
+ * bsr_requant_a -- gemm_dense_int8.rs, `requant_a_kernel` (first launch of
+ * `int8_gemm_faith2_prefill`).
+ *   a          [M, K] BF16 (raw uint16 bit patterns)
+ *   a_i8       [M, K] int8 out
+ *   a_scale_t  [K/32, ld] float out, block-major: the scale of row m, block b
+ *              is a_scale_t[b * ld + m], ld = bsr_a_scale_ld(M); entries
+ *              m >= M are not written
+ * Requirements: K > 0, K % 32 == 0; pointers 16-byte aligned.
+ */
+bsr_status bsr_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, int64_t m, int64_t k, void* stream);
+
+/*
+ * bsr_gemm -- gemm_dense_int8.rs, `faith2_kernel` (second launch of
+ * `int8_gemm_faith2_prefill`): the tcgen05 kind::i8 tensor-core GEMM with
+ * per-32-block rescale.
+ *   a_i8, a_scale_t  as written by bsr_requant_a (ld = bsr_a_scale_ld(M))
+ *   w_i8, w_scale    as written by bsr_requant_w
+ *   out              [M, N] BF16 out (uint16 bit patterns)
+ * Requirements: K % 128 == 0 (the W_scale row pitch must be a multiple of 16
+ * bytes for the tensor-memory-access copies); pointers 16-byte aligned.
+ */
+bsr_status bsr_gemm(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
+                    uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
+
+/*
+ * Scratch bytes bsr_proj needs for M rows (0 when M <= BSR_DECODE_MAX_M, or
+ * when K % 128 != 0, where the decode kernel serves every M): the int8
+ * activation codes (M*K bytes) then, 256-byte aligned, the block-major scales
+ * ((K/32) * bsr_a_scale_ld(M) floats) -- the caller-owned `a_i8_scratch` and
+ * `a_scale_scratch` of `int8_gemm_faith2_prefill`, in one buffer.
+ */
+size_t bsr_proj_scratch_bytes(int64_t m, int64_t k);
+
+/*
+ * bsr_proj -- gemm_dense_int8.rs, `int8_gemm_faith2_prefill`:
+ * out[M, N] = A[M, K] . W[N, K]^T from BF16 A and the requantised weight.
+ *   M <= BSR_DECODE_MAX_M: one launch of the decode kernel (CUDA cores,
+ *     activation requantisation fused, split over K across a warp); scratch
+ *     may be NULL.
+ *   M >  BSR_DECODE_MAX_M: bsr_requant_a into `scratch`, then bsr_gemm, both
+ *     on `stream`.  If K % 128 != 0 the decode kernel serves the rows instead
+ *     (in chunks of 16 rows per CTA row).
+ *   scratch        device buffer of at least bsr_proj_scratch_bytes(M, K)
+ *                  bytes, 256-byte aligned; contents are overwritten
+ * Requirements: K > 0, K % 32 == 0; a, w_i8, w_scale 16-byte aligned; out
+ * 2-byte aligned.
+ */
+bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m, int64_t n,
+                    int64_t k, void* scratch, size_t scratch_bytes, void* stream);
+
+/*
+ * bsr_decode -- the decode kernel of bsr_proj for any M (activation rows in
+ * groups of up to 16 per CTA row), exposed so both paths can be run on the
+ * same shapes.  No scratch.  Requirements as bsr_proj.
+ */
+bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                      int64_t n, int64_t k, void* stream);
+
+/*
+ * bsr_gemm_partials -- bsr_gemm that also writes every block partial
+ * P[m, n, b] (int32, [M, N, K/32]) exactly as the tensor cores produced it,
+ * for bit-exact checks.  Test use; slow.
+ */
+bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
+                             uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSR_H_ */

@@ -1,0 +1,97 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every function include/bsr.h declares with the binding's signatures, and
+rejects bad arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_scaled_precision_requant_b200 as bsr
+from block_scaled_precision_requant_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bsr.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return bsr.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bsr_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_what_binding_wraps():
+    assert _declared() == sorted(name for name, _, _ in bsr.SIGNATURES)
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+        assert ctypes.cast(getattr(L, name), ctypes.c_void_p).value
+
+
+def test_abi_version(L):
+    assert bsr.abi_version() == 1
+
+
+def test_scratch_and_ld(L):
+    assert bsr.a_scale_ld(1) == 4 and bsr.a_scale_ld(4) == 4 and bsr.a_scale_ld(4095) == 4096
+    assert bsr.proj_scratch_bytes(16, 4096) == 0  # decode path needs none
+    assert bsr.proj_scratch_bytes(17, 96) == 0  # K % 128 != 0: decode kernel serves it
+    m, k = 4095, 8192
+    codes = (m * k + 255) // 256 * 256
+    assert bsr.proj_scratch_bytes(m, k) == codes + (k // 32) * 4096 * 4
+
+
+P = ctypes.c_void_p
+
+
+def _fake(addr):
+    return P(addr)
+
+
+def test_shape_errors_before_launch(L):
+    s = L.bsr_proj(_fake(256), _fake(256), _fake(256), _fake(256), 4, 8, 48, None, 0, None)
+    assert s == 3 and "multiple of 32" in bsr.last_error()
+    assert L.bsr_gemm(_fake(256), _fake(256), _fake(256), _fake(256), _fake(256), 256, 256, 96, None) == 3
+    assert L.bsr_requant_w(_fake(256), _fake(256), ctypes.c_float(1.0), _fake(256), _fake(256), 4, 0, None) == 3
+
+
+def test_invalid_and_alignment_errors(L):
+    assert L.bsr_proj(None, _fake(256), _fake(256), _fake(256), 4, 8, 64, None, 0, None) == 1
+    assert L.bsr_proj(_fake(256), _fake(256), _fake(256), _fake(256), -1, 8, 64, None, 0, None) == 1
+    assert L.bsr_requant_a(_fake(264), _fake(256), _fake(256), 4, 64, None) == 2
+    assert L.bsr_gemm(_fake(256), _fake(256), _fake(256), _fake(256), _fake(257), 256, 256, 128, None) == 2
+    assert L.bsr_gemm_partials(_fake(256), _fake(256), _fake(256), _fake(256), _fake(256), None, 4, 4, 128,
+                               None) == 1
+
+
+def test_scratch_errors(L):
+    m, k = 64, 256
+    need = L.bsr_proj_scratch_bytes(m, k)
+    assert need > 0
+    assert L.bsr_proj(_fake(256), _fake(256), _fake(256), _fake(256), m, 8, k, None, 0, None) == 4
+    assert L.bsr_proj(_fake(256), _fake(256), _fake(256), _fake(256), m, 8, k, _fake(256), need - 1, None) == 4
+    assert L.bsr_proj(_fake(256), _fake(256), _fake(256), _fake(256), m, 8, k, _fake(272), need, None) == 2
+
+
+def test_empty_is_noop(L):
+    # M == 0 or N == 0 returns OK without touching any pointer or device
+    assert L.bsr_proj(None, None, None, None, 0, 8, 64, None, 0, None) == 0
+    assert L.bsr_proj(None, None, None, None, 4, 0, 64, None, 0, None) == 0
+    assert L.bsr_requant_w(None, None, ctypes.c_float(1.0), None, None, 0, 64, None) == 0
+    assert L.bsr_requant_a(None, None, None, 0, 64, None) == 0
+    assert L.bsr_gemm(None, None, None, None, None, 0, 4, 128, None) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(bsr, "_lib", None)
+    monkeypatch.setattr(bsr, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        bsr.lib()
