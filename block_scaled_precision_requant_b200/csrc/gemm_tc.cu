@@ -20,11 +20,14 @@
 //               scales by 2^49 and flags stages whose scales fall outside the
 //               exponent window of the fast epilogue.
 //   warps 4-11  epilogue: two warps per 32-lane quarter of tensor memory,
-//               64 activation columns each.
+//               64 activation columns each, read in the 16x256b fragment
+//               layout (4 weight rows x 2 adjacent columns per 8 columns).
 //
 // Epilogue arithmetic (per element and block, exact up to one rounding in
 // each of two FMAs):
-//   Tensor memory is preloaded with the integer 2^19 before every MMA, so the
+//   Every K block is two MMAs into the same buffer: first a u8 x u8 MMA of
+//   two constant tiles of 128s with accumulation off (32*128*128 = 2^19),
+//   then the s8 x s8 MMA of the data with accumulation on, so the
 //   accumulator holds P' = P + 2^19, which lies in [8160, 1040416] because
 //   |P| <= 32*127*127 = 516128 < 2^19.  Read as a float32 bit pattern, P' is
 //   the subnormal P' * 2^-149 exactly.  With W = w_scale * 2^100 and
@@ -58,9 +61,9 @@ constexpr int THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 // Register split: launched with 384 x 168 = 64512 registers; the control
 // warpgroup (warps 0-3) drops to 40 and the two epilogue warpgroups rise to
-// 224: 128 x 40 + 256 x 224 = 62464 <= 64512.
-constexpr int CTRL_REGS = 56;
-constexpr int EPI_REGS = 216;
+// 232: 128 x 40 + 256 x 232 = 64512.
+constexpr int CTRL_REGS = 40;
+constexpr int EPI_REGS = 232;
 static_assert(128 * CTRL_REGS + 256 * EPI_REGS <= THREADS * 168, "register split exceeds the launch allocation");
 
 constexpr int W_TILE = BN * KS;             // 16384
@@ -72,8 +75,12 @@ constexpr int OFF_A = W_TILE;
 constexpr int OFF_WS = W_TILE + A_TILE;
 constexpr int OFF_AS = OFF_WS + WS_TILE;
 
-constexpr uint32_t kBias = 1u << 19;
+constexpr uint32_t kBias = 1u << 19;  // = 32 * 128 * 128
 constexpr uint32_t kIdesc = idesc_i8(BN, BM);
+// u8 x u8 variant of the same shape, for the bias MMA
+constexpr uint32_t kIdescBias = kIdesc & ~((7u << 7) | (7u << 10));
+constexpr int CONST_TILE = BN * KS;  // 16 KB of 0x80 bytes: the bias MMA's operands
+static_assert(TBUF == KBS, "tensor-memory buffer index equals the K block index within a stage");
 
 struct Ctrl {
   uint64_t full[STAGES];
@@ -86,7 +93,7 @@ struct Ctrl {
   int abort_flag;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl);
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + CONST_TILE + sizeof(Ctrl);
 
 __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
@@ -96,9 +103,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const __grid_constant__ CUtensorMap tm_ws, const __grid_constant__ CUtensorMap tm_as,
                 __nv_bfloat16* __restrict__ out, int32_t* __restrict__ partials, int* __restrict__ status, int m,
                 int n, int k, int n_tiles, int m_tiles, int m_fastest) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(smem + (size_t)STAGES * STAGE_BYTES);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte-swizzled tiles, keeping the pointer
+  // derived from the shared array so accesses stay shared-space loads
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* const_tile = smem + (size_t)STAGES * STAGE_BYTES;
+  Ctrl* ctrl = reinterpret_cast<Ctrl*>(const_tile + CONST_TILE);
   volatile int* abort_flag = &ctrl->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -131,6 +141,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
+  for (int i = threadIdx.x; i < CONST_TILE / 16; i += THREADS)
+    reinterpret_cast<uint4*>(const_tile)[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -175,6 +188,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
+      const uint64_t c_desc = smem_desc_k_sw128(smem_u32(const_tile));
       uint32_t it = 0, g = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         for (int ks = 0; ks < kstages; ++ks, ++it) {
@@ -189,6 +203,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int buf = g % TBUF;
             if (!mbar_wait(&ctrl->tempty[buf], (g / TBUF) & 1, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
             tc_fence_after();
+            // D = 2^19 (constant u8 tiles of 128s, accumulate off), then D += A x B
+            mma_i8(tmem_base + buf * BM, c_desc, c_desc, kIdescBias, 0u);
             mma_i8(tmem_base + buf * BM, smem_desc_k_sw128(a_base + kb * 32), smem_desc_k_sw128(b_base + kb * 32),
                    kIdesc, 1u);
             tc_commit(&ctrl->tfull[buf]);
@@ -245,108 +261,197 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     setmaxnreg_inc<EPI_REGS>();
     // ---------------------------------------------------------------- epilogue
-    const int q = warp & 3;                    // tensor-memory lane quarter
-    const int hc = (warp - EPI_WARP0) >> 2;    // column half: 0 or 1
-    const int n_local = q * 32 + lane;
-    const uint32_t t_lane = (uint32_t)(q * 32) << 16;
-    const uint32_t col0 = (uint32_t)(hc * 64);
+    // Warp (quarter q, half hc) owns tensor-memory lanes 32q..32q+31 (weight
+    // rows) and columns 64hc..64hc+63 (activation rows).  It reads them with
+    // two 16x256b loads, so thread t holds weight rows 32q + t/4 + {0,8,16,24}
+    // and, per 8-column group j, the adjacent columns 8j + 2(t%4) + {0,1}:
+    // one 8-byte load of two activation scales then serves 8 elements.
+    // The four K blocks of a stage are unrolled (buffer = barrier = kb), and
+    // the next block's tensor-memory load is in flight while the current one
+    // is rescaled.
+    const int q = warp & 3;
+    const int hc = (warp - EPI_WARP0) >> 2;
+    const int t4 = lane >> 2;
+    const int tc = (lane & 3) * 2;
+    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(hc * 64);
+    const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const uint32_t smem_base = smem_u32(smem);
+    const uint32_t ws_off = OFF_WS + (uint32_t)((q * 32 + t4) * KBS) * 4u;  // + kb*4 + i*(8*KBS*4)
+    const uint32_t as_off = OFF_AS + (uint32_t)(hc * 64 + tc) * 4u;         // + kb*BM*4 + j*32
 
-    // preload the bias into every buffer slice this warp owns
-#pragma unroll
-    for (int b = 0; b < TBUF; ++b) tmem_st_x64_const(tmem_base + t_lane + b * BM + col0, kBias);
-    tc_wait_st();
-    tc_fence_before();
-    __syncwarp();
+    // open the tensor-memory ring
     if (lane == 0)
       for (int b = 0; b < TBUF; ++b) mbar_arrive(&ctrl->tempty[b]);
 
-    uint32_t it = 0, g = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      int n0, m0;
-      tile_coords(tile, n0, m0);
-      float2 acc[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = make_float2(0.0f, 0.0f);
+    float2 acc[4][8];
+    uint32_t pa0[32], pa1[32], pb0[32], pb1[32];
 
-      for (int ks = 0; ks < kstages; ++ks, ++it) {
-        const int s = it % STAGES;
-        const uint32_t r = it / STAGES;
-        if (!mbar_wait(&ctrl->prep[s], r & 1, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) goto epi_done;
-        const uint8_t* st = smem + (size_t)s * STAGE_BYTES;
-        const float* ws_row = reinterpret_cast<const float*>(st + OFF_WS) + n_local * KBS;
-        const int exotic = ctrl->exotic[s];
-        const float* as_stage = reinterpret_cast<const float*>(st + OFF_AS);
-#pragma unroll 1
-        for (int kb = 0; kb < KBS; ++kb, ++g) {
-          const int buf = g % TBUF;
-          if (!mbar_wait(&ctrl->tfull[buf], (g / TBUF) & 1, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) goto epi_done;
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + t_lane + buf * BM + col0;
-          uint32_t p[64];
-          tmem_ld_x64(taddr, p);
-          tmem_st_x64_const(taddr, kBias);
-          tc_wait_ld();
-          tc_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctrl->tempty[buf]);
+    // load block kb's partials (buffer kb) once its MMA has landed
+    auto tload = [&](int kb, uint32_t parity, uint32_t (&d0)[32], uint32_t (&d1)[32]) -> bool {  // kb: buffer
+      if (!mbar_wait(&ctrl->tfull[kb], parity, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
+      tc_fence_after();
+      tmem_ld_16x256b_x8(tl + kb * BM, d0);
+      tmem_ld_16x256b_x8(tl + kb * BM + (16u << 16), d1);
+      return true;
+    };
+    // after the load has landed, hand the buffer back to the MMA
+    auto trelease = [&](int kb) {
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctrl->tempty[kb]);
+    };
 
-          const float* arow = as_stage + kb * BM + col0;
-          const float wsb = ws_row[kb];
-          if (!exotic) {
-            const float W = wsb * 0x1p100f;
-            const float c = -(W * 0x1p-130f);
-            const float2 W2 = make_float2(W, W);
-            const float2 c2 = make_float2(c, c);
+    // Rescale 8-column groups j0..j0+3 of the current block.
+    auto rescale = [&](uint32_t st_addr, int kb, int exotic, int j0, const float (&wsr)[4],
+                       const uint32_t (&c0)[32], const uint32_t (&c1)[32]) {
+      const uint32_t aa = st_addr + as_off + (uint32_t)kb * (BM * 4u);
+      if (!exotic) {
+        float W[4], C[4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float4 a4 = reinterpret_cast<const float4*>(arow)[j];
-              const float2 u0 = __ffma2_rn(f2(p[4 * j], p[4 * j + 1]), W2, c2);
-              const float2 u1 = __ffma2_rn(f2(p[4 * j + 2], p[4 * j + 3]), W2, c2);
-              acc[2 * j] = __ffma2_rn(u0, make_float2(a4.x, a4.y), acc[2 * j]);
-              acc[2 * j + 1] = __ffma2_rn(u1, make_float2(a4.z, a4.w), acc[2 * j + 1]);
-            }
-          } else {
+        for (int i = 0; i < 4; ++i) {
+          W[i] = wsr[i] * 0x1p100f;
+          C[i] = -(W[i] * 0x1p-130f);
+        }
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float4 a4 = reinterpret_cast<const float4*>(arow)[j];
-              const float u0 = __fmul_rn(__int2float_rn((int)p[4 * j] - (int)kBias), wsb);
-              const float u1 = __fmul_rn(__int2float_rn((int)p[4 * j + 1] - (int)kBias), wsb);
-              const float u2 = __fmul_rn(__int2float_rn((int)p[4 * j + 2] - (int)kBias), wsb);
-              const float u3 = __fmul_rn(__int2float_rn((int)p[4 * j + 3] - (int)kBias), wsb);
-              acc[2 * j].x = __fmaf_rn(u0, a4.x, acc[2 * j].x);
-              acc[2 * j].y = __fmaf_rn(u1, a4.y, acc[2 * j].y);
-              acc[2 * j + 1].x = __fmaf_rn(u2, a4.z, acc[2 * j + 1].x);
-              acc[2 * j + 1].y = __fmaf_rn(u3, a4.w, acc[2 * j + 1].y);
-            }
+        for (int j = j0; j < j0 + 4; ++j) {
+          const float2 a2 = lds_f32x2(aa + (uint32_t)j * 32u);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t* pp = (i < 2) ? c0 : c1;
+            const int o = 4 * j + 2 * (i & 1);
+            float2 u;
+            u.x = __fmaf_rn(__uint_as_float(pp[o]), W[i], C[i]);
+            u.y = __fmaf_rn(__uint_as_float(pp[o + 1]), W[i], C[i]);
+            acc[i][j] = __ffma2_rn(u, a2, acc[i][j]);
           }
-          if constexpr (DUMP) {
-            const int nn = n0 + n_local;
-            const int b = ks * KBS + kb;
-            if (nn < n) {
+        }
+      } else {
 #pragma unroll
-              for (int c = 0; c < 64; ++c) {
-                const int mm = m0 + (int)col0 + c;
-                if (mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)p[c] - (int)kBias;
-              }
+        for (int j = j0; j < j0 + 4; ++j) {
+          const float2 a2 = lds_f32x2(aa + (uint32_t)j * 32u);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t* pp = (i < 2) ? c0 : c1;
+            const int o = 4 * j + 2 * (i & 1);
+            const float ux = __fmul_rn(__int2float_rn((int)pp[o] - (int)kBias), wsr[i]);
+            const float uy = __fmul_rn(__int2float_rn((int)pp[o + 1] - (int)kBias), wsr[i]);
+            acc[i][j].x = __fmaf_rn(ux, a2.x, acc[i][j].x);
+            acc[i][j].y = __fmaf_rn(uy, a2.y, acc[i][j].y);
+          }
+        }
+      }
+    };
+
+    // Zero-instruction scheduling fence: every accumulator flows through an
+    // empty volatile asm, so a block's FMAs complete before the next
+    // tensor-memory load (volatile asm) is issued and no register set is kept
+    // alive twice.
+    auto load_ws = [&](uint32_t st_addr, int kb, float (&wsr)[4]) {
+      const uint32_t wa = st_addr + ws_off + (uint32_t)kb * 4u;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wsr[i] = lds_f32(wa + (uint32_t)i * (8u * KBS * 4u));
+    };
+
+    auto acc_fence = [&]() {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        asm volatile(""
+                     : "+f"(acc[i][0].x), "+f"(acc[i][0].y), "+f"(acc[i][1].x), "+f"(acc[i][1].y),
+                       "+f"(acc[i][2].x), "+f"(acc[i][2].y), "+f"(acc[i][3].x), "+f"(acc[i][3].y),
+                       "+f"(acc[i][4].x), "+f"(acc[i][4].y), "+f"(acc[i][5].x), "+f"(acc[i][5].y),
+                       "+f"(acc[i][6].x), "+f"(acc[i][6].y), "+f"(acc[i][7].x), "+f"(acc[i][7].y));
+    };
+
+    auto dump = [&](int n0, int m0, int b, const uint32_t (&c0)[32], const uint32_t (&c1)[32]) {
+      if constexpr (DUMP) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int nn = n0 + q * 32 + t4 + 8 * i;
+          const uint32_t* pp = (i < 2) ? c0 : c1;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int mm = m0 + hc * 64 + 8 * j + tc + e;
+              if (nn < n && mm < m)
+                partials[((size_t)mm * n + nn) * nb + b] = (int)pp[4 * j + 2 * (i & 1) + e] - (int)kBias;
             }
           }
         }
+      }
+    };
+
+    // Block g of this CTA's sequence (tiles x K blocks): buffer/barrier
+    // g & 3 (= K block within the stage), stage counter g >> 2.
+    const int nbk = kstages * KBS;
+    const int total = my_tiles * nbk;
+    int tile = blockIdx.x, n0 = 0, m0 = 0, kbt = 0;
+    tile_coords(tile, n0, m0);
+    uint32_t st_addr = smem_base;
+    int exotic = 0;
+    float wsr[4];
+
+    auto step = [&](int g, uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t (&x0)[32], uint32_t (&x1)[32]) -> bool {
+      const int kb = g & (KBS - 1);
+      const uint32_t itg = (uint32_t)g >> 2;  // global stage counter
+      const int s = (int)(itg % STAGES);
+      const bool has_next = g + 1 < total;
+      if (kb == 0) {
+        if (!mbar_wait(&ctrl->prep[s], (itg / STAGES) & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
+        st_addr = smem_base + (uint32_t)s * STAGE_BYTES;
+        exotic = ctrl->exotic[s];
+      }
+      if (kbt == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+      }
+      load_ws(st_addr, kb, wsr);
+      rescale(st_addr, kb, exotic, 0, wsr, c0, c1);
+      // next block: same stage (phase itg & 1) or the next stage's block 0
+      if (has_next && !tload((g + 1) & (KBS - 1), ((uint32_t)(g + 1) >> 2) & 1u, x0, x1)) return false;
+      rescale(st_addr, kb, exotic, 4, wsr, c0, c1);
+      dump(n0, m0, kbt, c0, c1);
+      if (kb == KBS - 1) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->empty[s]);
       }
-      // tile end: write BF16; a warp's 32 lanes write 64 contiguous bytes per row
-      {
-        const int nn = n0 + n_local;
-        if (nn < n) {
+      if (++kbt == nbk) {
+        // tile end: write BF16 out[m][n]; the tile origin passes through a
+        // volatile move so the store addresses are formed here only
+        int nr, mr;
+        asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + t4));
+        asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + hc * 64 + tc));
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int mm = m0 + (int)col0 + 2 * j;
-            if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(acc[j].x);
-            if (mm + 1 < m) out[(size_t)(mm + 1) * n + nn] = __float2bfloat16_rn(acc[j].y);
+        for (int i = 0; i < 4; ++i) {
+          const int nn = nr + 8 * i;
+          if (nn < n) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int mm = mr + 8 * j;
+              if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(acc[i][j].x);
+              if (mm + 1 < m) out[(size_t)(mm + 1) * n + nn] = __float2bfloat16_rn(acc[i][j].y);
+            }
           }
         }
+        kbt = 0;
+        tile += gridDim.x;
+        tile_coords(tile, n0, m0);
       }
+      if (has_next) trelease((g + 1) & (KBS - 1));
+      return true;
+    };
+
+    bool ok = true;
+    if (total > 0) {
+      ok = tload(0, 0u, pa0, pa1);
+      if (ok) trelease(0);
+    }
+    for (int g = 0; ok && g < total; g += 2) {
+      ok = step(g, pa0, pa1, pb0, pb1);
+      if (ok && g + 1 < total) ok = step(g + 1, pb0, pb1, pa0, pa1);
     }
   epi_done:;
   }
