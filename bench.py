@@ -1,0 +1,536 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled int8 projection on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  A *step* is one pass of the projection path
+over one batch of synthetic input with the requantised weight resident (the
+weight requantisation runs once, before timing, as the launcher page's
+``ensure_int8_weight`` does):
+
+* ``decode`` (M=1, N=K=4096, the default): one launch of the decode kernel
+  (activation requantisation fused, CUDA cores); metric HBM GB/s over the
+  algorithmic bytes N*K + N*K/8 + 2*M*K + 2*M*N.
+* ``ffn_up`` / ``ffn_down`` / ``square_ragged``: requant_a + tcgen05 GEMM;
+  metric TOPS = 2*M*N*K / step time (requantisation included).
+
+L2 is flushed (a 256 MiB device write) before every timed step, outside the
+per-step CUDA events; ``ms_per_step`` is the mean of the per-step event times.
+``e2e`` repeats the step through the public API with the activations copied
+in from pinned host memory and the output copied back inside the events.
+Under torchrun every rank runs the same workload on its own GPU (independent
+replicas: the path has no exchange step), timings are max-reduced over ranks.
+``--impl reference`` times the CPU oracle (oracle/) on the host cores on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+INT8_PER_BF16 = 2.0  # nominal dense int8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="decode", choices=["decode", "ffn_up", "ffn_down", "square_ragged"])
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-extra", action="store_true", help="skip the secondary prefill measurements")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
+    p.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline (profiling runs)")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (one process per GPU; timing max-reduced over ranks)
+# ---------------------------------------------------------------------------
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def dist_init(backend: str):
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def dist_barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def dist_max(values, device="cpu"):
+    """Element-wise max over ranks of a list of floats (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def dist_sum(values, device="cpu"):
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.cpu().tolist()
+
+
+def dist_finish():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# peaks, clocks, roofline
+# ---------------------------------------------------------------------------
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = [
+        ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+        ("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+        ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+        ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+        ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+        ("applications_clocks_setting", "nvmlClocksEventReasonApplicationsClocksSetting"),
+    ]
+
+    def __init__(self, pci_bus_id: str | None, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(pci_bus_id) if pci_bus_id else pynvml.nvmlDeviceGetHandleByIndex(0)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # no NVML: clocks stay unknown
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, const in self.REASONS:
+                    if r & getattr(nv, const, 0):
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        return {
+            "sm_mhz": float(statistics.median(self.samples)) if self.samples else None,
+            "sm_max_mhz": float(self.max_mhz) if self.max_mhz else None,
+            "reasons": sorted(self.reasons),
+            "samples": len(self.samples),
+        }
+
+
+def roofline(bound, achieved, peak, unit, traffic):
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": (achieved / peak) if peak else None, "traffic": traffic}
+
+
+def kernel_source_hash():
+    """Hash of the CUDA sources: stored ncu traffic counts are valid only for it."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_scaled_precision_requant_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def stored_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from profiles/dram_traffic.txt (lines:
+    ``<kernel> <workload> <source-hash> <bytes>``), or None when absent or
+    taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    src = kernel_source_hash()
+    for line in lines:
+        parts = line.split()
+        if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[2] == src:
+            return float(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# workloads
+# ---------------------------------------------------------------------------
+
+
+def workload_desc(wl):
+    m, n, k = wl.shape
+    return {"workload": f"{wl.name}: M={m} N={n} K={k} (NVFP4 weight, BF16 activations '{wl.act}')",
+            "m": m, "n": n, "k": k, "seed": wl.seed,
+            "l2": "flushed before every timed step (256 MiB device write, outside the step events)"}
+
+
+def decode_bytes(m, n, k):
+    """Algorithmic HBM bytes of one decode step: int8 weight, its F32 scales
+    (4 B per 32), BF16 activations in, BF16 outputs out."""
+    return n * k + n * (k // 32) * 4 + 2 * m * k + 2 * m * n
+
+
+def prefill_ops(m, n, k):
+    return 2 * m * n * k
+
+
+class Gpu:
+    """Device state of one workload: requantised weight resident in HBM."""
+
+    def __init__(self, name, device):
+        import torch
+
+        from block_scaled_precision_requant_b200 import synth
+
+        import block_scaled_precision_requant_b200 as bsr
+
+        self.torch, self.bsr = torch, bsr
+        self.wl = synth.WORKLOADS[name]
+        d = synth.make_workload(name)
+        self.host = d
+        m, n, k = self.wl.shape
+        self.dev = device
+        wp = torch.from_numpy(d["w_packed"]).to(device)
+        we = torch.from_numpy(d["w_e4m3"]).to(device)
+        self.w_i8, self.w_s = bsr.requant_w(wp, we, float(d["scale2"]))
+        self.wp, self.we = wp, we
+        self.a = torch.from_numpy(d["a_bits"].view(np.int16)).view(torch.bfloat16).to(device)
+        self.out = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+        need = bsr.proj_scratch_bytes(m, k)
+        self.scratch = torch.empty((max(need, 1),), dtype=torch.uint8, device=device)
+        if m > bsr.DECODE_MAX_M:
+            self.a_i8, self.a_st = bsr.requant_a(self.a)
+        self.flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=device)
+        self.a_host = torch.from_numpy(d["a_bits"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.out_host = torch.empty((m, n), dtype=torch.bfloat16).pin_memory()
+        torch.cuda.synchronize()
+
+    def step(self):
+        self.bsr.proj(self.a, self.w_i8, self.w_s, self.out, self.scratch if self.scratch.numel() > 1 else None)
+
+    def step_e2e(self):
+        self.a.copy_(self.a_host, non_blocking=True)
+        self.step()
+        self.out_host.copy_(self.out, non_blocking=True)
+
+    def launches_per_step(self):
+        m, _, k = self.wl.shape
+        return 1 if (m <= self.bsr.DECODE_MAX_M or k % 128) else 2
+
+    def timed(self, fn, steps, warmup, events_inside=None):
+        """Per-step CUDA-event times (ms) of fn, L2 flushed before each step.
+        events_inside(i) may return (start, end) events of the dominant kernel."""
+        torch = self.torch
+        for _ in range(warmup):
+            self.flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        dist_barrier()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            self.flush.zero_()
+            ev[i][0].record()
+            fn()
+            ev[i][1].record()
+        torch.cuda.synchronize()
+        dist_barrier()
+        torch.cuda.synchronize()
+        return [s.elapsed_time(e) for s, e in ev]
+
+    def timed_gemm_only(self, steps, warmup):
+        """Events around the tensor-core GEMM alone (its own launch, same stream)."""
+        bsr = self.bsr
+        fn = lambda: bsr.gemm(self.a_i8, self.a_st, self.w_i8, self.w_s, self.out)
+        return self.timed(fn, steps, warmup)
+
+    def timed_requant_a_only(self, steps, warmup):
+        bsr = self.bsr
+        fn = lambda: bsr.requant_a(self.a, self.a_i8, self.a_st)
+        return self.timed(fn, steps, warmup)
+
+    def timed_requant_w_only(self, steps, warmup):
+        bsr = self.bsr
+        fn = lambda: bsr.requant_w(self.wp, self.we, float(self.host["scale2"]), self.w_i8, self.w_s)
+        return self.timed(fn, steps, warmup)
+
+    def check_status(self):
+        st = self.bsr.device_status()
+        if st != 0:
+            raise RuntimeError(f"device status word {st}: a pipeline wait timed out")
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# ---------------------------------------------------------------------------
+
+
+class OracleRunner:
+    """Times the CPU oracle on a bounded sample of a workload.  The weight
+    requantisation runs once, outside the timing (as on the GPU)."""
+
+    def __init__(self, name):
+        import oracle
+        from block_scaled_precision_requant_b200 import synth
+
+        self.oracle = oracle
+        self.wl = synth.WORKLOADS[name]
+        d = synth.make_workload(name)
+        m, n, k = self.wl.shape
+        self.w_i8, self.w_s = oracle.requant_w(d["w_packed"], d["w_e4m3"], d["scale2"], k)
+        self.a = d["a_bits"]
+        self.rows = synth.sample_rows(m, min(m, 64), self.wl.seed)
+
+    def sample_step(self, nrows):
+        """Oracle projection of `nrows` sampled rows; returns seconds."""
+        t0 = time.perf_counter()
+        self.oracle.proj_rows(self.a[self.rows[:nrows]], self.w_i8, self.w_s)
+        return time.perf_counter() - t0
+
+    def per_row_seconds(self, budget_s):
+        """Mean oracle seconds per activation row over a sample bounded by budget_s."""
+        done, spent = 0, 0.0
+        while spent < budget_s and done < 1000:
+            spent += self.sample_step(1)
+            done += 1
+        return spent / done, done
+
+
+def units_per_step(wl):
+    m, n, k = wl.shape
+    if m <= 16:
+        return decode_bytes(m, n, k) / 1e9, "GB/s", "int8 block-scaled proj HBM GB/s (M=1 decode, incl. requant)"
+    return prefill_ops(m, n, k) / 1e12, "TOPS", "int8 block-scaled proj TOPS (prefill, incl. requant)"
+
+
+def cpu_baseline(name, budget_s):
+    r = OracleRunner(name)
+    per_row, rows = r.per_row_seconds(budget_s)
+    units, unit, _ = units_per_step(r.wl)
+    step_s = per_row * r.wl.m
+    sample = (f"{rows} oracle projection(s) of one activation row each against the full requantised weight, "
+              f"timed on the host; step time = per-row time x M={r.wl.m}" + (" (extrapolated)" if r.wl.m > 1 else ""))
+    return {"value": units / step_s, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample,
+            "ms_per_step": step_s * 1e3}
+
+
+def reference_main(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from block_scaled_precision_requant_b200 import synth
+
+    wl = synth.WORKLOADS[args.workload]
+    r = OracleRunner(args.workload)
+    units, unit, metric = units_per_step(wl)
+    for _ in range(args.warmup):
+        r.sample_step(1)
+    t = [r.sample_step(1) for _ in range(args.steps)]
+    step_s = float(np.mean(t)) * wl.m
+    value = units / step_s
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded generator)", "impl": "reference",
+            "config": workload_desc(wl),
+            "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                             "sample": f"each step: the oracle on 1 of {len(r.rows)} sampled activation rows against the "
+                                       f"full requantised weight; step time = per-row time x M={wl.m}"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+
+def mean_ms(times):
+    return float(np.mean(times))
+
+
+def prefill_extra(name, device, steps, warmup, peaks):
+    """Secondary measurement of one prefill workload (rank-local)."""
+    g = Gpu(name, device)
+    m, n, k = g.wl.shape
+    ops = prefill_ops(m, n, k)
+    t_step = mean_ms(g.timed(g.step, steps, warmup))
+    t_gemm = mean_ms(g.timed_gemm_only(steps, warmup))
+    t_ra = mean_ms(g.timed_requant_a_only(steps, warmup))
+    t_rw = mean_ms(g.timed_requant_w_only(steps, warmup))
+    g.check_status()
+    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    res = {
+        "shape": [m, n, k],
+        "tops_incl_requant": ops / t_step / 1e9,
+        "gemm_tops": ops / t_gemm / 1e9,
+        "gemm_frac_of_int8_peak": ops / t_gemm / 1e9 / int8_peak,
+        "requant_a_gbs": m * k * 3.125 / t_ra / 1e6,
+        "requant_w_gbs": n * k * 1.6875 / t_rw / 1e6,
+        "ms": {"step": t_step, "gemm": t_gemm, "requant_a": t_ra, "requant_w": t_rw},
+    }
+    del g
+    import torch
+
+    torch.cuda.empty_cache()
+    return res
+
+
+def gpu_main(args):
+    import torch
+
+    rank, world, local = dist_init("nccl")
+    if not torch.cuda.is_available():
+        raise RuntimeError("no CUDA device: the GPU arm has no CPU fallback")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    props = torch.cuda.get_device_properties(dev)
+    pci = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+    peaks, peak_src = load_peaks()
+
+    g = Gpu(args.workload, dev)
+    wl = g.wl
+    m, n, k = wl.shape
+    units, unit, metric = units_per_step(wl)
+    decode = m <= g.bsr.DECODE_MAX_M
+
+    with ClockSampler(pci) as clk:
+        t_steps = g.timed(g.step, args.steps, args.warmup)
+    t_e2e = g.timed(g.step_e2e, args.steps, args.warmup)
+    if decode:
+        t_kernel = t_steps  # the step is one launch of the decode kernel
+        kernel = "decode_kernel"
+    else:
+        t_kernel = g.timed_gemm_only(args.steps, args.warmup)
+        kernel = "gemm_kernel"
+    t_rw = g.timed_requant_w_only(min(args.steps, 20), args.warmup)
+    g.check_status()
+
+    ms_step, ms_e2e, ms_kernel, ms_rw = dist_max(
+        [mean_ms(t_steps), mean_ms(t_e2e), mean_ms(t_kernel), mean_ms(t_rw)], device="cuda" if world > 1 else "cpu")
+    value = world * units / (ms_step / 1e3)
+    e2e_value = world * units / (ms_e2e / 1e3)
+    if decode:
+        rl = roofline("hbm", decode_bytes(m, n, k) / (ms_kernel / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s",
+                      stored_traffic(kernel, wl.name))
+    else:
+        rl = roofline("tensor", prefill_ops(m, n, k) / (ms_kernel / 1e3) / 1e12,
+                      peaks["bf16_tflops"] * INT8_PER_BF16, "TOPS", stored_traffic(kernel, wl.name))
+    rl["kernel"] = kernel
+    rl["peak_source"] = (f"{peak_src} (HBM copy)" if decode else
+                         f"{peak_src} bf16 cuBLAS burst x {INT8_PER_BF16:g} (nominal int8/bf16 ratio)")
+
+    line = {
+        "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
+        "data": "synthetic (seeded generator; no dataset or trained weights)",
+        "config": {**workload_desc(wl), "parallelism": f"replicas x{world} (no exchange step)"},
+        "roofline": rl,
+        "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": 2 * m * k, "d2h_bytes_per_step": 2 * m * n,
+                "ms_per_step": ms_e2e},
+        "gpu_launches": g.launches_per_step() * args.steps,
+        "clocks": clk.summary(),
+        "requant_w": {"gbs": n * k * 1.6875 / (ms_rw / 1e3) / 1e9, "ms": ms_rw,
+                      "frac_of_hbm": n * k * 1.6875 / (ms_rw / 1e3) / 1e9 / peaks["hbm_gbs"]},
+    }
+    del g
+    torch.cuda.empty_cache()
+    if not args.no_extra and world == 1:
+        extra = {}
+        for name in ("ffn_up", "ffn_down", "square_ragged"):
+            if name != args.workload:
+                extra[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks)
+        line["prefill"] = extra
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    dist_finish()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return reference_main(args)
+    return gpu_main(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

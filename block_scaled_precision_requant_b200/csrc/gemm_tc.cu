@@ -453,7 +453,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = step(g, pa0, pa1, pb0, pb1);
       if (ok && g + 1 < total) ok = step(g + 1, pb0, pb1, pa0, pa1);
     }
-  epi_done:;
   }
 
   tc_fence_before();

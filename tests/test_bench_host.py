@@ -1,0 +1,91 @@
+"""Host-side logic of bench.py on CPU: the multi-rank timing reduction over
+gloo (world size 2), the JSON line of the reference arm, and the stored
+traffic lookup."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, q):
+    os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    bench.dist_init("gloo")
+    # each rank reports its own step times; the job time is the max over ranks
+    mine = [1.0 + rank, 2.0 - rank, 5.0 * (rank + 1)]
+    mx = bench.dist_max(mine)
+    sm = bench.dist_sum([1.0])
+    bench.dist_barrier()
+    bench.dist_finish()
+    q.put((rank, mx, sm))
+
+
+def test_dist_max_over_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in procs]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, mx, sm in res:
+        assert mx == [2.0, 2.0, 10.0]
+        assert sm == [2.0]
+
+
+def test_single_rank_reduction_is_identity():
+    assert bench.dist_max([3.0, 4.0]) == [3.0, 4.0]
+
+
+def test_reference_arm_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_reference_arm_non_zero_rank_exits_quietly():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1"],
+                         capture_output=True, text=True, timeout=120, cwd=ROOT, env=env)
+    assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_units_and_bytes():
+    from block_scaled_precision_requant_b200 import synth
+
+    assert bench.decode_bytes(1, 4096, 4096) == 18890752
+    u, unit, _ = bench.units_per_step(synth.WORKLOADS["ffn_up"])
+    assert unit == "TOPS" and abs(u - 2 * 2048 * 14336 * 4096 / 1e12) < 1e-9
+
+
+def test_stored_traffic_requires_matching_source(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    src = bench.kernel_source_hash()
+    (prof / "dram_traffic.txt").write_text(f"decode_kernel decode {src} 123\ndecode_kernel decode deadbeef 7\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: src)
+    assert bench.stored_traffic("decode_kernel", "decode") == 123.0
+    assert bench.stored_traffic("gemm_kernel", "decode") is None
