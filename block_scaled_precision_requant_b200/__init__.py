@@ -72,6 +72,7 @@ SIGNATURES = [
     ("bsr_proj", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_decode", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_gemm_partials", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("bsr_proj_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
 ]
 
 

@@ -173,6 +173,16 @@ bsr_status check_proj_args(const uint16_t* a, const int8_t* w_i8, const float* w
 
 }  // namespace
 
+namespace bsr {
+bsr_status report(bsr_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+}  // namespace bsr
+
 extern "C" {
 
 int bsr_abi_version(void) { return BSR_ABI_VERSION; }

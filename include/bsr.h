@@ -33,7 +33,9 @@
  *     which rows of a stacked weight are launched together.
  *
  * Memory: every pointer is a device pointer (except where noted) owned by the
- * caller; the library never allocates device memory.  All arrays are dense
+ * caller; no call allocates device memory (the library's own device storage
+ * is a status word and the bsr_proj_noalloc array, both reserved when the
+ * library's GPU code is loaded).  All arrays are dense
  * row-major.  Every call is asynchronous on `stream` (a cudaStream_t, NULL =
  * the legacy default stream) and returns before the kernels finish.
  *
@@ -167,6 +169,30 @@ bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scal
  */
 bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
                              uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream);
+
+/* Size of the device array bsr_proj_noalloc uses as its scratch: 16 MiB,
+ * enough for M*K + (K/32)*round_up(M,4)*4 <= 16 MiB (e.g. M=2048, K=4096 or
+ * M=3584, K=4096; not M=4095, K=8192). */
+#define BSR_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * bsr_proj_noalloc -- bsr_proj for callers that cannot allocate device memory
+ * at call time (a runtime that plans all device memory ahead and passes only
+ * inputs and outputs, or code where cudaMalloc, which synchronises the
+ * device, is not allowed).  No counterpart on the launcher pages: it is this
+ * library's addition.  Same arguments, results and errors as bsr_proj without
+ * the scratch pair; the activation codes and scales live in a device array
+ * inside the library (BSR_NOALLOC_SCRATCH_BYTES, held on every GPU that loads
+ * the library until the process exits).  Calls that need more return
+ * BSR_ESCRATCH without launching.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress, with that device current);
+ * make that first call before any stream capture.  Every call reuses the same
+ * array: calls that may overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller.  Allocates
+ * nothing, never calls cudaMalloc or cudaFree.
+ */
+bsr_status bsr_proj_noalloc(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                            int64_t n, int64_t k, void* stream);
 
 #ifdef __cplusplus
 }
