@@ -159,8 +159,8 @@ bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_sca
   if ((st = device_info(d)) != BSR_OK) return st;
   const int mr = bsr::decode_rows_per_cta((int)m, (int)k, d.smem_optin);
   if (mr == 0) return fail(BSR_ESHAPE, "K=%lld too large for the decode kernel's shared memory", (long long)k);
-  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, as_stream(stream),
-                                        d.num_sms),
+  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, d.status, d.smem_optin,
+                                        as_stream(stream), d.num_sms),
                      "decode launch");
 }
 

@@ -21,6 +21,7 @@ enum : int {
   DEV_ERR_TIMEOUT_MMA = 2,
   DEV_ERR_TIMEOUT_EPI = 4,
   DEV_ERR_TIMEOUT_PREP = 8,
+  DEV_ERR_TIMEOUT_DECODE = 16,
 };
 
 // 1 s of waiting on one barrier is far beyond any legal schedule here.
@@ -132,6 +133,16 @@ __device__ __forceinline__ void tma_load_2d_hint(void* dst, const CUtensorMap* m
       "%4}], [%2], %5;" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(policy)
       : "memory");
+}
+
+// Contiguous global -> shared copy by the bulk-copy (TMA) engine, completing
+// `bytes` of transaction count on `bar`.  Addresses 16-byte aligned, size a
+// multiple of 16.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 // ---------------------------------------------------------------------------

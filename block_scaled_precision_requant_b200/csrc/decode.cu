@@ -8,10 +8,13 @@
 // l, l+32, ...) and the 32 lane sums are added in a fixed xor tree, so an
 // output's bits depend only on K, never on M, N or the launch grid.
 //
-// Each CTA re-quantises the activation rows it serves into shared memory (a
-// few KB read from L2), after issuing its first weight loads so the HBM
-// latency overlaps with that work.  The int8 codes and scales match the
-// standalone requant_a kernel bit for bit (same rule, same quant.cuh).
+// Memory: one warp per weight row.  Each warp streams its row (and, when the
+// row pitch allows, the row's scales) into its own shared-memory slot with a
+// single bulk copy issued at kernel start, so the whole weight is in flight
+// at once without holding registers.  Meanwhile the CTA requantises the
+// activation rows into shared memory (same rule and code as requant_a, so
+// the codes match it bit for bit), then each warp waits for its row and
+// forms the block dot products from shared memory.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -20,8 +23,10 @@
 
 namespace bsr {
 
-constexpr int kDecodeWarps = 8;
-constexpr int kDecodeUnroll = 4;  // 32-blocks per lane in flight
+// Warps (= weight rows in flight) per CTA at most: 32 for one or two
+// activation rows, 8 for more (their per-row register arrays grow).
+template <int MR>
+constexpr int decode_max_warps() { return MR <= 2 ? 32 : 8; }
 
 __device__ __forceinline__ void bf16x8_to_f32_d(const uint4& v, float (&x)[8]) {
   x[0] = __uint_as_float(v.x << 16);
@@ -47,58 +52,105 @@ __device__ __forceinline__ int dot32(const uint4& w0, const uint4& w1, const uin
   return p;
 }
 
-// MR: activation rows per CTA (compile time, >= rows actually present).
-// Shared memory: codes [MR][K] int8, then scales [MR][K/32] f32.
-template <int MR>
-__global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const uint16_t* __restrict__ a,
-                                                                    const int8_t* __restrict__ w_i8,
-                                                                    const float* __restrict__ w_scale,
-                                                                    __nv_bfloat16* __restrict__ out, int m, int n,
-                                                                    int k) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  const int nb = k >> 5;
-  int8_t* s_codes = reinterpret_cast<int8_t*>(smem);
-  float* s_scale = reinterpret_cast<float*>(smem + (size_t)MR * k);
+// Shared-memory layout of one CTA (byte offsets).
+struct DecodeSmem {
+  uint32_t codes, ascale, wrow, wscale, bars, abort_flag, total;
+  uint32_t wrow_bytes, wscale_bytes;  // per warp
+  uint32_t chunks;                    // 1 KB weight chunks per row (one 32-block per lane)
+};
 
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline DecodeSmem decode_smem_layout(int mr, int k, int nwarps, bool scale_bulk) {
+  DecodeSmem L;
+  const uint32_t nb = (uint32_t)k / 32;
+  L.codes = 0;
+  L.ascale = align_up((uint32_t)mr * (uint32_t)k, 16);
+  L.wrow_bytes = (uint32_t)k;
+  L.wscale_bytes = scale_bulk ? nb * 4 : 0;
+  L.wrow = align_up(L.ascale + (uint32_t)mr * nb * 4, 128);
+  L.wscale = L.wrow + (uint32_t)nwarps * L.wrow_bytes;
+  L.chunks = (nb + 31) / 32;
+  L.bars = align_up(L.wscale + (uint32_t)nwarps * L.wscale_bytes, 8);
+  L.abort_flag = L.bars + (uint32_t)nwarps * L.chunks * 8;
+  L.total = L.abort_flag + 16;
+  return L;
+}
+
+// MR: activation rows per CTA (compile time, >= rows actually present).
+template <int MR>
+__global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
+    decode_kernel(const uint16_t* __restrict__ a, const int8_t* __restrict__ w_i8, const float* __restrict__ w_scale,
+                  __nv_bfloat16* __restrict__ out, int m, int n, int k, int scale_bulk, int* __restrict__ status) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int nb = k >> 5;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const DecodeSmem L = decode_smem_layout(MR, k, nwarps, scale_bulk != 0);
+  int8_t* s_codes = reinterpret_cast<int8_t*>(smem + L.codes);
+  float* s_scale = reinterpret_cast<float*>(smem + L.ascale);
+  int8_t* s_w = reinterpret_cast<int8_t*>(smem + L.wrow + (uint32_t)warp * L.wrow_bytes);
+  float* s_ws = reinterpret_cast<float*>(smem + L.wscale + (uint32_t)warp * L.wscale_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + (size_t)warp * L.chunks;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.abort_flag);
+
   const int m0 = blockIdx.y * MR;
   const int rows = min(MR, m - m0);
+  int row = blockIdx.x * nwarps + warp;
+  const int row_step = gridDim.x * nwarps;
 
-  int row = blockIdx.x * kDecodeWarps + warp;
-  const int row_step = gridDim.x * kDecodeWarps;
+  // Launched with programmatic stream serialisation: the grid may be
+  // scheduled while the previous kernel on the stream drains.  Wait for that
+  // kernel to complete (and its writes to be visible) before the first
+  // global read, and let the next kernel be scheduled early in turn.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // First weight tile of this warp's first row, issued before the activation pass.
-  uint4 wv[kDecodeUnroll][2];
-  float ws[kDecodeUnroll];
-  auto load_tile = [&](int r, int it) {
-#pragma unroll
-    for (int u = 0; u < kDecodeUnroll; ++u) {
-      const int b = (it * kDecodeUnroll + u) * 32 + lane;
-      if (r < n && b < nb) {
-        const uint4* src = reinterpret_cast<const uint4*>(w_i8 + (size_t)r * k + (size_t)b * 32);
-        wv[u][0] = __ldg(src);
-        wv[u][1] = __ldg(src + 1);
-        ws[u] = __ldg(w_scale + (size_t)r * nb + b);
-      } else {
-        wv[u][0] = wv[u][1] = make_uint4(0, 0, 0, 0);
-        ws[u] = 0.0f;
+  if (threadIdx.x == 0) *abort_flag = 0;
+  if (lane == 0) {
+    for (uint32_t c = 0; c < L.chunks; ++c) mbar_init(&bars[c], 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // A row goes out as 1 KB chunks (one 32-block per lane), each completing
+  // on its own barrier, so the first chunks can be consumed while the rest
+  // of the weight is still streaming.
+  auto issue_row = [&](int r) {
+    if (lane == 0 && r < n) {
+      for (uint32_t c = 0; c < L.chunks; ++c) {
+        const uint32_t blocks = min(32u, (uint32_t)nb - 32u * c);
+        const uint32_t wb = blocks * 32u, sb = L.wscale_bytes ? blocks * 4u : 0u;
+        mbar_arrive_expect_tx(&bars[c], wb + sb);
+        bulk_load(s_w + (size_t)c * 1024, w_i8 + (size_t)r * k + (size_t)c * 1024, wb, &bars[c]);
+        if (sb) bulk_load(s_ws + (size_t)c * 32, w_scale + (size_t)r * nb + (size_t)c * 32, sb, &bars[c]);
       }
     }
   };
-  load_tile(row, 0);
 
-  // Activation requantisation into shared memory: 4 lanes per 32-group.
+  // Activation requantisation into shared memory: 4 lanes per 32-group,
+  // 8 groups per warp per pass.  The first pass's activation loads go out
+  // before the weight copies so they are not queued behind the weight stream.
   {
     const int groups = MR * nb;
     const int sub = lane & 3;
-    for (int g0 = warp * 8; g0 < groups; g0 += kDecodeWarps * 8) {
+    auto load_act = [&](int g0) {
       const int g = g0 + (lane >> 2);
       const int r = g / nb;
       const int b = g - r * nb;
-      const bool valid = (g < groups) && (r < rows);
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (valid) v = __ldg(reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * k + (size_t)b * 32 + sub * 8));
+      if (g < groups && r < rows)
+        v = __ldg(reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * k + (size_t)b * 32 + sub * 8));
+      return v;
+    };
+    uint4 av = load_act(warp * 8);
+    issue_row(row);
+    for (int g0 = warp * 8; g0 < groups; g0 += nwarps * 8) {
+      const int g = g0 + (lane >> 2);
+      const int r = g / nb;
+      const int b = g - r * nb;
+      const uint4 v = av;
+      if (g0 + nwarps * 8 < groups) av = load_act(g0 + nwarps * 8);
       float x[8];
       bf16x8_to_f32_d(v, x);
       float amax = 0.0f;
@@ -119,36 +171,40 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const uint16_
   }
   __syncthreads();
 
-  // Lane l reads the two 16-byte halves of its block in the order h, 1-h with
-  // h = (l >> 2) & 1, so that each 8-lane phase of a 16-byte shared load hits
-  // eight distinct 16-byte bank groups.
+  // Lane l reads the two 16-byte halves of its 32-byte block in the order h,
+  // 1-h with h = (l >> 2) & 1, so each 8-lane phase of a 16-byte shared load
+  // hits eight distinct 16-byte bank groups.
   const int h = (lane >> 2) & 1;
-  const int iters = (nb + 32 * kDecodeUnroll - 1) / (32 * kDecodeUnroll);
-
+  uint32_t phase = 0;
+  bool aborted = false;
   for (; row < n; row += row_step) {
     float acc[MR];
 #pragma unroll
     for (int r = 0; r < MR; ++r) acc[r] = 0.0f;
-    for (int it = 0; it < iters; ++it) {
-      if (it > 0) load_tile(row, it);
+    for (int b = lane, c = 0; c < (int)L.chunks; b += 32, ++c) {
+      if (!mbar_wait(&bars[c], phase, abort_flag, status, DEV_ERR_TIMEOUT_DECODE)) {
+        aborted = true;
+        break;
+      }
+      if (b >= nb) continue;
+      const uint4* wsrc = reinterpret_cast<const uint4*>(s_w + (size_t)b * 32);
+      const uint4 w0 = wsrc[h];
+      const uint4 w1 = wsrc[1 - h];
+      const float wsb = L.wscale_bytes ? s_ws[b] : __ldg(w_scale + (size_t)row * nb + b);
 #pragma unroll
-      for (int u = 0; u < kDecodeUnroll; ++u) {
-        const int b = (it * kDecodeUnroll + u) * 32 + lane;
-        if (b < nb) {
-          const uint4 w0 = h ? wv[u][1] : wv[u][0];
-          const uint4 w1 = h ? wv[u][0] : wv[u][1];
-#pragma unroll
-          for (int r = 0; r < MR; ++r) {
-            const uint4* cs = reinterpret_cast<const uint4*>(s_codes + (size_t)r * k + (size_t)b * 32);
-            const uint4 a0 = cs[h];
-            const uint4 a1 = cs[1 - h];
-            const int p = dot32(w0, w1, a0, a1);
-            const float u_ = __fmul_rn((float)p, ws[u]);
-            acc[r] = __fmaf_rn(u_, s_scale[r * nb + b], acc[r]);
-          }
-        }
+      for (int r = 0; r < MR; ++r) {
+        const uint4* cs = reinterpret_cast<const uint4*>(s_codes + (size_t)r * k + (size_t)b * 32);
+        const int p = dot32(w0, w1, cs[h], cs[1 - h]);
+        const float u = __fmul_rn(__int2float_rn(p), wsb);
+        acc[r] = __fmaf_rn(u, s_scale[r * nb + b], acc[r]);
       }
     }
+    if (aborted) break;
+    phase ^= 1u;
+    // every lane has read the row slot: it may be refilled (async proxy)
+    __syncwarp();
+    fence_proxy_async_smem();
+    issue_row(row + row_step);
     // fixed-order reduction over the 32 lanes
 #pragma unroll
     for (int r = 0; r < MR; ++r) {
@@ -162,52 +218,81 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_kernel(const uint16_
       for (int r = 0; r < MR; ++r)
         if (r < rows) out[(size_t)(m0 + r) * n + row] = __float2bfloat16_rn(acc[r]);
     }
-    const int next = row + row_step;
-    if (next < n) load_tile(next, 0);
+  }
+  // A warp that gave up waiting may still have its copy in flight: wait for it
+  // once more, again bounded, so the CTA does not exit under a bulk copy.
+  if (aborted && lane == 0) {
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t c = 0; c < L.chunks; ++c)
+      while (!mbar_try_wait(&bars[c], phase) && globaltimer_ns() - t0 < kWaitLimitNs) {
+      }
   }
 }
 
-static size_t decode_smem(int mr, int k) { return (size_t)mr * k + (size_t)mr * (k / 32) * 4; }
+static bool decode_scale_bulk(int k) { return (k % 128) == 0; }
 
 // Rows per CTA: the largest power of two <= 16 that covers M and fits the
-// shared-memory budget.
+// shared-memory budget together with at least one weight-row slot.
 int decode_rows_per_cta(int m, int k, size_t smem_limit) {
   int mr = 1;
   while (mr < m && mr < 16) mr <<= 1;
-  while (mr > 1 && decode_smem(mr, k) > smem_limit) mr >>= 1;
-  if (decode_smem(mr, k) > smem_limit) return 0;
-  return mr;
+  auto fits = [&](int r) { return decode_smem_layout(r, k, 1, decode_scale_bulk(k)).total <= smem_limit; };
+  while (mr > 1 && !fits(mr)) mr >>= 1;
+  return fits(mr) ? mr : 0;
 }
 
 template <int MR>
 static cudaError_t launch_decode_t(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m,
-                                   int n, int k, cudaStream_t stream, int num_sms) {
-  const size_t smem = decode_smem(MR, k);
+                                   int n, int k, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
   auto kern = decode_kernel<MR>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool sb = decode_scale_bulk(k);
+  // Warps (= weight rows in flight) per CTA: spread the rows over all SMs,
+  // at most decode_max_warps<MR>() per CTA and as many row slots as fit in
+  // shared memory; beyond one CTA per SM the warps loop over rows.
+  constexpr int kMaxW = decode_max_warps<MR>();
+  int w = (int)((n + (long long)num_sms - 1) / num_sms);
+  w = w < 1 ? 1 : (w > kMaxW ? kMaxW : w);
+  while (w > 1 && decode_smem_layout(MR, k, w, sb).total > smem_limit) --w;
+  const size_t smem = decode_smem_layout(MR, k, w, sb).total;
+  // dynamic shared-memory limit granted so far, per device
+  static size_t granted[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecodeWarps * 32, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
-  long long gx = (n + kDecodeWarps - 1) / kDecodeWarps;
-  const long long cap = (long long)num_sms * per_sm;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (smem > granted[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    granted[dev] = smem;
+  }
   const int gy = (m + MR - 1) / MR;
-  if (gx * gy > cap) gx = (cap + gy - 1) / gy;
+  long long gx = (n + w - 1) / w;
+  if (gx * gy > num_sms) gx = ((long long)num_sms + gy - 1) / gy;
   if (gx < 1) gx = 1;
-  dim3 grid((unsigned)gx, (unsigned)gy);
-  kern<<<grid, kDecodeWarps * 32, smem, stream>>>(a, w_i8, w_scale, reinterpret_cast<__nv_bfloat16*>(out), m, n, k);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)gx, (unsigned)gy);
+  cfg.blockDim = dim3(w * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  e = cudaLaunchKernelEx(&cfg, kern, a, w_i8, w_scale, o, m, n, k, sb ? 1 : 0, status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
-                          int k, int mr, cudaStream_t stream, int num_sms) {
+                          int k, int mr, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
   switch (mr) {
-    case 1: return launch_decode_t<1>(a, w_i8, w_scale, out, m, n, k, stream, num_sms);
-    case 2: return launch_decode_t<2>(a, w_i8, w_scale, out, m, n, k, stream, num_sms);
-    case 4: return launch_decode_t<4>(a, w_i8, w_scale, out, m, n, k, stream, num_sms);
-    case 8: return launch_decode_t<8>(a, w_i8, w_scale, out, m, n, k, stream, num_sms);
-    case 16: return launch_decode_t<16>(a, w_i8, w_scale, out, m, n, k, stream, num_sms);
+    case 1: return launch_decode_t<1>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
+    case 2: return launch_decode_t<2>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
+    case 4: return launch_decode_t<4>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
+    case 8: return launch_decode_t<8>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
+    case 16: return launch_decode_t<16>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -475,16 +475,27 @@ cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, 
   // Sweep the smaller operand fastest so that it stays resident in L2 while
   // the larger one streams through once.
   const int m_fastest = ((long long)m <= (long long)n) ? 1 : 0;
-  cudaError_t e;
+  // the shared-memory opt-in is set once per device and kernel variant
+  static bool granted[64][2] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (partials) {
-    e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    if (!granted[dev][1]) {
+      e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      granted[dev][1] = true;
+    }
     gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(maps.w, maps.a, maps.ws, maps.as,
                                                              reinterpret_cast<__nv_bfloat16*>(out), partials,
                                                              status, m, n, k, n_tiles, m_tiles, m_fastest);
   } else {
-    e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    if (e != cudaSuccess) return e;
+    if (!granted[dev][0]) {
+      e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+      if (e != cudaSuccess) return e;
+      granted[dev][0] = true;
+    }
     gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(maps.w, maps.a, maps.ws, maps.as,
                                                               reinterpret_cast<__nv_bfloat16*>(out), nullptr,
                                                               status, m, n, k, n_tiles, m_tiles, m_fastest);
