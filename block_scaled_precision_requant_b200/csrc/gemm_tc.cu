@@ -15,10 +15,12 @@
 //   warp 0      TMA producer: per stage (4 K blocks = 128 bytes of K) the W
 //               and A tiles (128x128 bytes, 128-byte swizzle) and their
 //               scale tiles, into a 5-stage shared-memory ring.
-//   warp 1      tensor-memory allocation and the MMA issuer (one thread).
+//   warps 1, 3  MMA issuers (one thread each; K blocks 0,2 and 1,3 of a
+//               stage); warp 1 also allocates the tensor memory.
 //   warp 2      scale preparation: pre-multiplies the staged activation
-//               scales by 2^49 and flags stages whose scales fall outside the
-//               exponent window of the fast epilogue.
+//               scales by 2^49 and the weight scales by 2^100, or flags the
+//               stage when a scale falls outside the exponent window of the
+//               fast epilogue (the stage then keeps its scales as loaded).
 //   warps 4-11  epilogue: two warps per 32-lane quarter of tensor memory,
 //               64 activation columns each, read in the 16x256b fragment
 //               layout (4 weight rows x 2 adjacent columns per 8 columns).
@@ -42,6 +44,8 @@
 //   fma) for all its blocks.  Two FMAs per element run as packed f32x2 FMAs.
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -60,10 +64,10 @@ constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 // Register split: launched with 384 x 168 = 64512 registers; the control
-// warpgroup (warps 0-3) drops to 40 and the two epilogue warpgroups rise to
-// 232: 128 x 40 + 256 x 232 = 64512.
-constexpr int CTRL_REGS = 40;
-constexpr int EPI_REGS = 232;
+// warpgroup (warps 0-3) drops to 56 and the two epilogue warpgroups rise to
+// 224: 128 x 56 + 256 x 224 = 64512.
+constexpr int CTRL_REGS = 56;
+constexpr int EPI_REGS = 224;
 static_assert(128 * CTRL_REGS + 256 * EPI_REGS <= THREADS * 168, "register split exceeds the launch allocation");
 
 constexpr int W_TILE = BN * KS;             // 16384
@@ -120,7 +124,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctrl->full[s], 1);
-      mbar_init(&ctrl->empty[s], 1 + EPI_WARPS);
+      mbar_init(&ctrl->empty[s], 2 + EPI_WARPS);  // two MMA commits + the epilogue warps
       mbar_init(&ctrl->prep[s], 1);
       ctrl->exotic[s] = 0;
     }
@@ -185,11 +189,15 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     tma_done:;
     }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 3) {
     // ---------------------------------------------------------------- MMA
+    // Two issuing threads: warp 1 takes K blocks 0 and 2 of every stage,
+    // warp 3 blocks 1 and 3 (= tensor-memory buffers), so the per-block issue
+    // cost (two MMAs and a commit) is paid on two warps.
     if (lane == 0) {
       const uint64_t c_desc = smem_desc_k_sw128(smem_u32(const_tile));
-      uint32_t it = 0, g = 0;
+      const int kb0 = (warp == 1) ? 0 : 1;
+      uint32_t it = 0;
       for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
         for (int ks = 0; ks < kstages; ++ks, ++it) {
           const int s = it % STAGES;
@@ -199,15 +207,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t a_base = smem_u32(smem + (size_t)s * STAGE_BYTES);
           const uint32_t b_base = a_base + OFF_A;
 #pragma unroll
-          for (int kb = 0; kb < KBS; ++kb, ++g) {
-            const int buf = g % TBUF;
-            if (!mbar_wait(&ctrl->tempty[buf], (g / TBUF) & 1, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
+          for (int kb = kb0; kb < KBS; kb += 2) {
+            if (!mbar_wait(&ctrl->tempty[kb], it & 1, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
             tc_fence_after();
             // D = 2^19 (constant u8 tiles of 128s, accumulate off), then D += A x B
-            mma_i8(tmem_base + buf * BM, c_desc, c_desc, kIdescBias, 0u);
-            mma_i8(tmem_base + buf * BM, smem_desc_k_sw128(a_base + kb * 32), smem_desc_k_sw128(b_base + kb * 32),
+            mma_i8(tmem_base + kb * BM, c_desc, c_desc, kIdescBias, 0u);
+            mma_i8(tmem_base + kb * BM, smem_desc_k_sw128(a_base + kb * 32), smem_desc_k_sw128(b_base + kb * 32),
                    kIdesc, 1u);
-            tc_commit(&ctrl->tfull[buf]);
+            tc_commit(&ctrl->tfull[kb]);
           }
           tc_commit(&ctrl->empty[s]);
         }
@@ -224,23 +231,24 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait(&ctrl->full[s], r & 1, abort_flag, status, DEV_ERR_TIMEOUT_PREP)) goto prep_done;
         uint8_t* st = smem + (size_t)s * STAGE_BYTES;
         float4* as4 = reinterpret_cast<float4*>(st + OFF_AS);
-        const float4* ws4 = reinterpret_cast<const float4*>(st + OFF_WS);
-        float4 av[4];
+        float4* ws4 = reinterpret_cast<float4*>(st + OFF_WS);
+        float4 av[4], wv[4];
         bool bad = false;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           av[j] = as4[j * 32 + lane];
           bad |= !(av[j].x < 0x1p79f) | !(av[j].y < 0x1p79f) | !(av[j].z < 0x1p79f) | !(av[j].w < 0x1p79f);
-          const float4 w = ws4[j * 32 + lane];
-          const float wv[4] = {w.x, w.y, w.z, w.w};
+          wv[j] = ws4[j * 32 + lane];
+          const float w4[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
-            const float aw = fabsf(wv[t]);
+            const float aw = fabsf(w4[t]);
             bad |= !((aw == 0.0f) | ((aw >= 0x1p-77f) & (aw < 0x1p28f)));
           }
         }
         const bool exotic = __any_sync(0xFFFFFFFFu, bad);
         if (!exotic) {
+          // a_scale * 2^49 and W = w_scale * 2^100, both exact inside the window
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             float4 v = av[j];
@@ -249,6 +257,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             v.z *= 0x1p49f;
             v.w *= 0x1p49f;
             as4[j * 32 + lane] = v;
+            float4 w = wv[j];
+            w.x *= 0x1p100f;
+            w.y *= 0x1p100f;
+            w.z *= 0x1p100f;
+            w.w *= 0x1p100f;
+            ws4[j * 32 + lane] = w;
           }
         }
         if (lane == 0) ctrl->exotic[s] = exotic ? 1 : 0;
@@ -307,12 +321,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                        const uint32_t (&c0)[32], const uint32_t (&c1)[32]) {
       const uint32_t aa = st_addr + as_off + (uint32_t)kb * (BM * 4u);
       if (!exotic) {
-        float W[4], C[4];
+        // wsr holds W = w_scale * 2^100 here; C = -W * 2^-130
+        float C[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          W[i] = wsr[i] * 0x1p100f;
-          C[i] = -(W[i] * 0x1p-130f);
-        }
+        for (int i = 0; i < 4; ++i) C[i] = -(wsr[i] * 0x1p-130f);
 #pragma unroll
         for (int j = j0; j < j0 + 4; ++j) {
           const float2 a2 = lds_f32x2(aa + (uint32_t)j * 32u);
@@ -321,8 +333,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t* pp = (i < 2) ? c0 : c1;
             const int o = 4 * j + 2 * (i & 1);
             float2 u;
-            u.x = __fmaf_rn(__uint_as_float(pp[o]), W[i], C[i]);
-            u.y = __fmaf_rn(__uint_as_float(pp[o + 1]), W[i], C[i]);
+            u.x = __fmaf_rn(__uint_as_float(pp[o]), wsr[i], C[i]);
+            u.y = __fmaf_rn(__uint_as_float(pp[o + 1]), wsr[i], C[i]);
             acc[i][j] = __ffma2_rn(u, a2, acc[i][j]);
           }
         }
@@ -382,76 +394,82 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     };
 
-    // Block g of this CTA's sequence (tiles x K blocks): buffer/barrier
-    // g & 3 (= K block within the stage), stage counter g >> 2.
-    const int nbk = kstages * KBS;
-    const int total = my_tiles * nbk;
-    int tile = blockIdx.x, n0 = 0, m0 = 0, kbt = 0;
+    // Stage sequence of this CTA: stage counter itg (tiles x K stages), ring
+    // slot itg % STAGES; within a stage the four K blocks are unrolled, block
+    // kb in tensor-memory buffer kb (phase itg & 1), with the partials of
+    // even blocks in (pa0, pa1) and of odd blocks in (pb0, pb1).
+    const int total_st = my_tiles * kstages;
+    int tile = blockIdx.x, n0 = 0, m0 = 0, kst = 0;
     tile_coords(tile, n0, m0);
     uint32_t st_addr = smem_base;
     int exotic = 0;
-    float wsr[4];
+    uint32_t itg = 0;
 
-    auto step = [&](int g, uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t (&x0)[32], uint32_t (&x1)[32]) -> bool {
-      const int kb = g & (KBS - 1);
-      const uint32_t itg = (uint32_t)g >> 2;  // global stage counter
+    auto sub = [&](auto kbc, uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t (&x0)[32],
+                   uint32_t (&x1)[32]) -> bool {
+      constexpr int kb = decltype(kbc)::value;
       const int s = (int)(itg % STAGES);
-      const bool has_next = g + 1 < total;
-      if (kb == 0) {
-        if (!mbar_wait(&ctrl->prep[s], (itg / STAGES) & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
-        st_addr = smem_base + (uint32_t)s * STAGE_BYTES;
-        exotic = ctrl->exotic[s];
+      float wsr[4];
+      load_ws(st_addr, kb, wsr);
+      rescale(st_addr, kb, exotic, 0, wsr, c0, c1);
+      // next block: block kb+1 of this stage, or block 0 of the next stage
+      const bool has_next = (kb < KBS - 1) || (itg + 1 < (uint32_t)total_st);
+      if (has_next) {
+        const uint32_t par = (kb < KBS - 1) ? (itg & 1u) : ((itg + 1) & 1u);
+        if (!tload((kb + 1) & (KBS - 1), par, x0, x1)) return false;
       }
-      if (kbt == 0) {
+      rescale(st_addr, kb, exotic, 4, wsr, c0, c1);
+      dump(n0, m0, kst * KBS + kb, c0, c1);
+      if (kb == KBS - 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctrl->empty[s]);
+        if (++kst == kstages) {
+          // tile end: write BF16 out[m][n]; the tile origin passes through a
+          // volatile move so the store addresses are formed here only
+          int nr, mr;
+          asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + t4));
+          asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + hc * 64 + tc));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int nn = nr + 8 * i;
+            if (nn < n) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const int mm = mr + 8 * j;
+                if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(acc[i][j].x);
+                if (mm + 1 < m) out[(size_t)(mm + 1) * n + nn] = __float2bfloat16_rn(acc[i][j].y);
+              }
+            }
+          }
+          kst = 0;
+          tile += gridDim.x;
+          tile_coords(tile, n0, m0);
+        }
+      }
+      if (has_next) trelease((kb + 1) & (KBS - 1));
+      return true;
+    };
+
+    bool ok = true;
+    if (total_st > 0) {
+      ok = tload(0, 0u, pa0, pa1);
+      if (ok) trelease(0);
+    }
+    for (; ok && itg < (uint32_t)total_st; ++itg) {
+      const int s = (int)(itg % STAGES);
+      if (!mbar_wait(&ctrl->prep[s], (itg / STAGES) & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) break;
+      st_addr = smem_base + (uint32_t)s * STAGE_BYTES;
+      exotic = ctrl->exotic[s];
+      if (kst == 0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
           for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
       }
-      load_ws(st_addr, kb, wsr);
-      rescale(st_addr, kb, exotic, 0, wsr, c0, c1);
-      // next block: same stage (phase itg & 1) or the next stage's block 0
-      if (has_next && !tload((g + 1) & (KBS - 1), ((uint32_t)(g + 1) >> 2) & 1u, x0, x1)) return false;
-      rescale(st_addr, kb, exotic, 4, wsr, c0, c1);
-      dump(n0, m0, kbt, c0, c1);
-      if (kb == KBS - 1) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->empty[s]);
-      }
-      if (++kbt == nbk) {
-        // tile end: write BF16 out[m][n]; the tile origin passes through a
-        // volatile move so the store addresses are formed here only
-        int nr, mr;
-        asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + t4));
-        asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + hc * 64 + tc));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int nn = nr + 8 * i;
-          if (nn < n) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int mm = mr + 8 * j;
-              if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(acc[i][j].x);
-              if (mm + 1 < m) out[(size_t)(mm + 1) * n + nn] = __float2bfloat16_rn(acc[i][j].y);
-            }
-          }
-        }
-        kbt = 0;
-        tile += gridDim.x;
-        tile_coords(tile, n0, m0);
-      }
-      if (has_next) trelease((g + 1) & (KBS - 1));
-      return true;
-    };
-
-    bool ok = true;
-    if (total > 0) {
-      ok = tload(0, 0u, pa0, pa1);
-      if (ok) trelease(0);
-    }
-    for (int g = 0; ok && g < total; g += 2) {
-      ok = step(g, pa0, pa1, pb0, pb1);
-      if (ok && g + 1 < total) ok = step(g + 1, pb0, pb1, pa0, pa1);
+      ok = sub(std::integral_constant<int, 0>{}, pa0, pa1, pb0, pb1) &&
+           sub(std::integral_constant<int, 1>{}, pb0, pb1, pa0, pa1) &&
+           sub(std::integral_constant<int, 2>{}, pa0, pa1, pb0, pb1) &&
+           sub(std::integral_constant<int, 3>{}, pb0, pb1, pa0, pa1);
     }
   }
 
