@@ -22,8 +22,9 @@
 //               stage when a scale falls outside the exponent window of the
 //               fast epilogue (the stage then keeps its scales as loaded).
 //   warps 4-11  epilogue: two warps per 32-lane quarter of tensor memory,
-//               64 activation columns each, read in the 16x256b fragment
-//               layout (4 weight rows x 2 adjacent columns per 8 columns).
+//               64 activation columns each, read with 32x32b loads (one
+//               weight row per thread; this shape moves about three times
+//               the bytes per cycle of the 16x256b one).
 //
 // Epilogue arithmetic (per element and block, exact up to one rounding in
 // each of two FMAs):
@@ -276,36 +277,34 @@ __global__ void __launch_bounds__(THREADS, 1)
     setmaxnreg_inc<EPI_REGS>();
     // ---------------------------------------------------------------- epilogue
     // Warp (quarter q, half hc) owns tensor-memory lanes 32q..32q+31 (weight
-    // rows) and columns 64hc..64hc+63 (activation rows).  It reads them with
-    // two 16x256b loads, so thread t holds weight rows 32q + t/4 + {0,8,16,24}
-    // and, per 8-column group j, the adjacent columns 8j + 2(t%4) + {0,1}:
-    // one 8-byte load of two activation scales then serves 8 elements.
-    // The four K blocks of a stage are unrolled (buffer = barrier = kb), and
-    // the next block's tensor-memory load is in flight while the current one
-    // is rescaled.
+    // rows) and columns 64hc..64hc+63 (activation rows), read with one
+    // 32x32b.x64 load per block: thread t holds weight row 32q + t and the
+    // 64 activation rows of its half.  Its weight scales for the four blocks
+    // of a stage are one 16-byte load; the activation scales, the same for the
+    // whole warp, are broadcast 16-byte loads.  The four K blocks of a stage
+    // are unrolled (buffer = barrier = kb), and the next block's tensor-memory
+    // load is in flight while the second half of the current block is
+    // rescaled.
     const int q = warp & 3;
     const int hc = (warp - EPI_WARP0) >> 2;
-    const int t4 = lane >> 2;
-    const int tc = (lane & 3) * 2;
     const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(hc * 64);
     const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const uint32_t smem_base = smem_u32(smem);
-    const uint32_t ws_off = OFF_WS + (uint32_t)((q * 32 + t4) * KBS) * 4u;  // + kb*4 + i*(8*KBS*4)
-    const uint32_t as_off = OFF_AS + (uint32_t)(hc * 64 + tc) * 4u;         // + kb*BM*4 + j*32
+    const uint32_t ws_off = OFF_WS + (uint32_t)((q * 32 + lane) * KBS) * 4u;  // [n][kb]
+    const uint32_t as_off = OFF_AS + (uint32_t)(hc * 64) * 4u;                // + kb*BM*4 + c*4
 
     // open the tensor-memory ring
     if (lane == 0)
       for (int b = 0; b < TBUF; ++b) mbar_arrive(&ctrl->tempty[b]);
 
-    float2 acc[4][8];
-    uint32_t pa0[32], pa1[32], pb0[32], pb1[32];
+    float2 acc[32];  // acc[c/2] = columns (c, c+1)
+    uint32_t pa[64], pb[64];
 
     // load block kb's partials (buffer kb) once its MMA has landed
-    auto tload = [&](int kb, uint32_t parity, uint32_t (&d0)[32], uint32_t (&d1)[32]) -> bool {  // kb: buffer
+    auto tload = [&](int kb, uint32_t parity, uint32_t (&d)[64]) -> bool {
       if (!mbar_wait(&ctrl->tfull[kb], parity, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
       tc_fence_after();
-      tmem_ld_16x256b_x8(tl + kb * BM, d0);
-      tmem_ld_16x256b_x8(tl + kb * BM + (16u << 16), d1);
+      tmem_ld_x64(tl + kb * BM, d);
       return true;
     };
     // after the load has landed, hand the buffer back to the MMA
@@ -316,79 +315,45 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (lane == 0) mbar_arrive(&ctrl->tempty[kb]);
     };
 
-    // Rescale 8-column groups j0..j0+3 of the current block.
-    auto rescale = [&](uint32_t st_addr, int kb, int exotic, int j0, const float (&wsr)[4],
-                       const uint32_t (&c0)[32], const uint32_t (&c1)[32]) {
-      const uint32_t aa = st_addr + as_off + (uint32_t)kb * (BM * 4u);
+    // Rescale columns c0..c0+31 of the current block (W, C: this thread's
+    // weight-row constants; exotic stages use the plain convert-multiply-fma).
+    auto rescale = [&](uint32_t aa, int exotic, int c0, float W, const uint32_t (&p)[64]) {
       if (!exotic) {
-        // wsr holds W = w_scale * 2^100 here; C = -W * 2^-130
-        float C[4];
+        const float C = -(W * 0x1p-130f);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) C[i] = -(wsr[i] * 0x1p-130f);
-#pragma unroll
-        for (int j = j0; j < j0 + 4; ++j) {
-          const float2 a2 = lds_f32x2(aa + (uint32_t)j * 32u);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t* pp = (i < 2) ? c0 : c1;
-            const int o = 4 * j + 2 * (i & 1);
-            float2 u;
-            u.x = __fmaf_rn(__uint_as_float(pp[o]), wsr[i], C[i]);
-            u.y = __fmaf_rn(__uint_as_float(pp[o + 1]), wsr[i], C[i]);
-            acc[i][j] = __ffma2_rn(u, a2, acc[i][j]);
-          }
+        for (int c = c0; c < c0 + 32; c += 4) {
+          const float4 a4 = lds_f32x4(aa + (uint32_t)c * 4u);
+          float2 u0, u1;
+          u0.x = __fmaf_rn(__uint_as_float(p[c]), W, C);
+          u0.y = __fmaf_rn(__uint_as_float(p[c + 1]), W, C);
+          u1.x = __fmaf_rn(__uint_as_float(p[c + 2]), W, C);
+          u1.y = __fmaf_rn(__uint_as_float(p[c + 3]), W, C);
+          acc[c / 2] = __ffma2_rn(u0, make_float2(a4.x, a4.y), acc[c / 2]);
+          acc[c / 2 + 1] = __ffma2_rn(u1, make_float2(a4.z, a4.w), acc[c / 2 + 1]);
         }
       } else {
 #pragma unroll
-        for (int j = j0; j < j0 + 4; ++j) {
-          const float2 a2 = lds_f32x2(aa + (uint32_t)j * 32u);
+        for (int c = c0; c < c0 + 32; c += 4) {
+          const float4 a4 = lds_f32x4(aa + (uint32_t)c * 4u);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t* pp = (i < 2) ? c0 : c1;
-            const int o = 4 * j + 2 * (i & 1);
-            const float ux = __fmul_rn(__int2float_rn((int)pp[o] - (int)kBias), wsr[i]);
-            const float uy = __fmul_rn(__int2float_rn((int)pp[o + 1] - (int)kBias), wsr[i]);
-            acc[i][j].x = __fmaf_rn(ux, a2.x, acc[i][j].x);
-            acc[i][j].y = __fmaf_rn(uy, a2.y, acc[i][j].y);
+          for (int e = 0; e < 4; ++e) {
+            const float u = __fmul_rn(__int2float_rn((int)p[c + e] - (int)kBias), W);
+            float& dst = (e & 1) ? acc[(c + e) / 2].y : acc[(c + e) / 2].x;
+            dst = __fmaf_rn(u, av[e], dst);
           }
         }
       }
     };
 
-    // Zero-instruction scheduling fence: every accumulator flows through an
-    // empty volatile asm, so a block's FMAs complete before the next
-    // tensor-memory load (volatile asm) is issued and no register set is kept
-    // alive twice.
-    auto load_ws = [&](uint32_t st_addr, int kb, float (&wsr)[4]) {
-      const uint32_t wa = st_addr + ws_off + (uint32_t)kb * 4u;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) wsr[i] = lds_f32(wa + (uint32_t)i * (8u * KBS * 4u));
-    };
-
-    auto acc_fence = [&]() {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        asm volatile(""
-                     : "+f"(acc[i][0].x), "+f"(acc[i][0].y), "+f"(acc[i][1].x), "+f"(acc[i][1].y),
-                       "+f"(acc[i][2].x), "+f"(acc[i][2].y), "+f"(acc[i][3].x), "+f"(acc[i][3].y),
-                       "+f"(acc[i][4].x), "+f"(acc[i][4].y), "+f"(acc[i][5].x), "+f"(acc[i][5].y),
-                       "+f"(acc[i][6].x), "+f"(acc[i][6].y), "+f"(acc[i][7].x), "+f"(acc[i][7].y));
-    };
-
-    auto dump = [&](int n0, int m0, int b, const uint32_t (&c0)[32], const uint32_t (&c1)[32]) {
+    auto dump = [&](int n0, int m0, int b, const uint32_t (&p)[64]) {
       if constexpr (DUMP) {
+        const int nn = n0 + q * 32 + lane;
+        if (nn < n) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int nn = n0 + q * 32 + t4 + 8 * i;
-          const uint32_t* pp = (i < 2) ? c0 : c1;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int mm = m0 + hc * 64 + 8 * j + tc + e;
-              if (nn < n && mm < m)
-                partials[((size_t)mm * n + nn) * nb + b] = (int)pp[4 * j + 2 * (i & 1) + e] - (int)kBias;
-            }
+          for (int c = 0; c < 64; ++c) {
+            const int mm = m0 + hc * 64 + c;
+            if (mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)p[c] - (int)kBias;
           }
         }
       }
@@ -397,48 +362,45 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Stage sequence of this CTA: stage counter itg (tiles x K stages), ring
     // slot itg % STAGES; within a stage the four K blocks are unrolled, block
     // kb in tensor-memory buffer kb (phase itg & 1), with the partials of
-    // even blocks in (pa0, pa1) and of odd blocks in (pb0, pb1).
+    // even blocks in pa and of odd blocks in pb.
     const int total_st = my_tiles * kstages;
     int tile = blockIdx.x, n0 = 0, m0 = 0, kst = 0;
     tile_coords(tile, n0, m0);
     uint32_t st_addr = smem_base;
     int exotic = 0;
+    float4 wst = make_float4(0.f, 0.f, 0.f, 0.f);
     uint32_t itg = 0;
 
-    auto sub = [&](auto kbc, uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t (&x0)[32],
-                   uint32_t (&x1)[32]) -> bool {
+    auto sub = [&](auto kbc, uint32_t (&cur)[64], uint32_t (&nxt)[64]) -> bool {
       constexpr int kb = decltype(kbc)::value;
       const int s = (int)(itg % STAGES);
-      float wsr[4];
-      load_ws(st_addr, kb, wsr);
-      rescale(st_addr, kb, exotic, 0, wsr, c0, c1);
+      const float W = (kb == 0) ? wst.x : (kb == 1) ? wst.y : (kb == 2) ? wst.z : wst.w;
+      const uint32_t aa = st_addr + as_off + (uint32_t)kb * (BM * 4u);
+      rescale(aa, exotic, 0, W, cur);
       // next block: block kb+1 of this stage, or block 0 of the next stage
       const bool has_next = (kb < KBS - 1) || (itg + 1 < (uint32_t)total_st);
       if (has_next) {
         const uint32_t par = (kb < KBS - 1) ? (itg & 1u) : ((itg + 1) & 1u);
-        if (!tload((kb + 1) & (KBS - 1), par, x0, x1)) return false;
+        if (!tload((kb + 1) & (KBS - 1), par, nxt)) return false;
       }
-      rescale(st_addr, kb, exotic, 4, wsr, c0, c1);
-      dump(n0, m0, kst * KBS + kb, c0, c1);
+      rescale(aa, exotic, 32, W, cur);
+      dump(n0, m0, kst * KBS + kb, cur);
       if (kb == KBS - 1) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctrl->empty[s]);
         if (++kst == kstages) {
-          // tile end: write BF16 out[m][n]; the tile origin passes through a
-          // volatile move so the store addresses are formed here only
+          // tile end: write BF16 out[m][n] (lanes = consecutive n); the
+          // tile origin passes through a volatile move so the store
+          // addresses are formed here only
           int nr, mr;
-          asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + t4));
-          asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + hc * 64 + tc));
+          asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + lane));
+          asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + hc * 64));
+          if (nr < n) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int nn = nr + 8 * i;
-            if (nn < n) {
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const int mm = mr + 8 * j;
-                if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(acc[i][j].x);
-                if (mm + 1 < m) out[(size_t)(mm + 1) * n + nn] = __float2bfloat16_rn(acc[i][j].y);
-              }
+            for (int c = 0; c < 64; c += 2) {
+              const int mm = mr + c;
+              if (mm < m) out[(size_t)mm * n + nr] = __float2bfloat16_rn(acc[c / 2].x);
+              if (mm + 1 < m) out[(size_t)(mm + 1) * n + nr] = __float2bfloat16_rn(acc[c / 2].y);
             }
           }
           kst = 0;
@@ -452,7 +414,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     bool ok = true;
     if (total_st > 0) {
-      ok = tload(0, 0u, pa0, pa1);
+      ok = tload(0, 0u, pa);
       if (ok) trelease(0);
     }
     for (; ok && itg < (uint32_t)total_st; ++itg) {
@@ -460,16 +422,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(&ctrl->prep[s], (itg / STAGES) & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) break;
       st_addr = smem_base + (uint32_t)s * STAGE_BYTES;
       exotic = ctrl->exotic[s];
+      wst = lds_f32x4(st_addr + ws_off);
       if (kst == 0) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+        for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.0f, 0.0f);
       }
-      ok = sub(std::integral_constant<int, 0>{}, pa0, pa1, pb0, pb1) &&
-           sub(std::integral_constant<int, 1>{}, pb0, pb1, pa0, pa1) &&
-           sub(std::integral_constant<int, 2>{}, pa0, pa1, pb0, pb1) &&
-           sub(std::integral_constant<int, 3>{}, pb0, pb1, pa0, pa1);
+      ok = sub(std::integral_constant<int, 0>{}, pa, pb) && sub(std::integral_constant<int, 1>{}, pb, pa) &&
+           sub(std::integral_constant<int, 2>{}, pa, pb) && sub(std::integral_constant<int, 3>{}, pb, pa);
     }
   }
 
