@@ -311,14 +311,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto trelease = [&](int kb) {
       tc_wait_ld();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctrl->tempty[kb]);
+      mbar_arrive_lane0(&ctrl->tempty[kb], lane);
     };
 
     // Rescale columns c0..c0+31 of the current block (W, C: this thread's
     // weight-row constants; exotic stages use the plain convert-multiply-fma).
-    auto rescale = [&](uint32_t aa, int exotic, int c0, float W, const uint32_t (&p)[64]) {
-      if (!exotic) {
+    // The choice is a template parameter: a stage runs one of two fully
+    // unrolled code paths, with no branch inside the per-block loop.
+    auto rescale = [&](auto exc, uint32_t aa, int c0, float W, const uint32_t (&p)[64]) {
+      if constexpr (!decltype(exc)::value) {
         const float C = -(W * 0x1p-130f);
 #pragma unroll
         for (int c = c0; c < c0 + 32; c += 4) {
@@ -371,23 +372,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     float4 wst = make_float4(0.f, 0.f, 0.f, 0.f);
     uint32_t itg = 0;
 
-    auto sub = [&](auto kbc, uint32_t (&cur)[64], uint32_t (&nxt)[64]) -> bool {
+    auto sub = [&](auto kbc, auto exc, uint32_t (&cur)[64], uint32_t (&nxt)[64]) -> bool {
       constexpr int kb = decltype(kbc)::value;
       const int s = (int)(itg % STAGES);
       const float W = (kb == 0) ? wst.x : (kb == 1) ? wst.y : (kb == 2) ? wst.z : wst.w;
       const uint32_t aa = st_addr + as_off + (uint32_t)kb * (BM * 4u);
-      rescale(aa, exotic, 0, W, cur);
+      rescale(exc, aa, 0, W, cur);
       // next block: block kb+1 of this stage, or block 0 of the next stage
       const bool has_next = (kb < KBS - 1) || (itg + 1 < (uint32_t)total_st);
       if (has_next) {
         const uint32_t par = (kb < KBS - 1) ? (itg & 1u) : ((itg + 1) & 1u);
         if (!tload((kb + 1) & (KBS - 1), par, nxt)) return false;
       }
-      rescale(aa, exotic, 32, W, cur);
+      rescale(exc, aa, 32, W, cur);
       dump(n0, m0, kst * KBS + kb, cur);
       if (kb == KBS - 1) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->empty[s]);
+        mbar_arrive_lane0(&ctrl->empty[s], lane);
         if (++kst == kstages) {
           // tile end: write BF16 out[m][n] (lanes = consecutive n); the
           // tile origin passes through a volatile move so the store
@@ -427,8 +427,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.0f, 0.0f);
       }
-      ok = sub(std::integral_constant<int, 0>{}, pa, pb) && sub(std::integral_constant<int, 1>{}, pb, pa) &&
-           sub(std::integral_constant<int, 2>{}, pa, pb) && sub(std::integral_constant<int, 3>{}, pb, pa);
+      using K0 = std::integral_constant<int, 0>;
+      using K1 = std::integral_constant<int, 1>;
+      using K2 = std::integral_constant<int, 2>;
+      using K3 = std::integral_constant<int, 3>;
+      if (!exotic) {
+        const std::false_type fast;
+        ok = sub(K0{}, fast, pa, pb) && sub(K1{}, fast, pb, pa) && sub(K2{}, fast, pa, pb) && sub(K3{}, fast, pb, pa);
+      } else {
+        const std::true_type slow;
+        ok = sub(K0{}, slow, pa, pb) && sub(K1{}, slow, pb, pa) && sub(K2{}, slow, pa, pb) && sub(K3{}, slow, pb, pa);
+      }
     }
   }
 
