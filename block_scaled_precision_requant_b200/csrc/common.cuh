@@ -279,6 +279,18 @@ __device__ __forceinline__ void tmem_ld_16x128b_x16(uint32_t taddr, uint32_t (&r
       : "r"(taddr));
 }
 
+// 16 lanes x 128 bits, repeated 8 times along the columns (32 columns):
+// thread t holds r[2k] = (lane t/4, column t%4 + 4k) and
+// r[2k+1] = (lane t/4 + 8, same column), k = 0..7.
+__device__ __forceinline__ void tmem_ld_16x128b_x8(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x128b.x8.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.16x256b.x8.b32 "

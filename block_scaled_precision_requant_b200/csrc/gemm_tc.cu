@@ -11,7 +11,7 @@
 // such buffers lets the MMA of block b+1..b+3 run while the epilogue warps
 // rescale block b into float32 register accumulators.
 //
-// Warp roles (384 threads, one CTA per SM, persistent over tiles):
+// Warp roles (640 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: per stage (4 K blocks = 128 bytes of K) the W
 //               and A tiles (128x128 bytes, 128-byte swizzle) and their
 //               scale tiles, into a 5-stage shared-memory ring.
@@ -21,10 +21,9 @@
 //               scales by 2^49 and the weight scales by 2^100, or flags the
 //               stage when a scale falls outside the exponent window of the
 //               fast epilogue (the stage then keeps its scales as loaded).
-//   warps 4-11  epilogue: two warps per 32-lane quarter of tensor memory,
-//               64 activation columns each, read with 32x32b loads (one
-//               weight row per thread; this shape moves about three times
-//               the bytes per cycle of the 16x256b one).
+//   warps 4-19  epilogue: four warps per 32-lane quarter of tensor memory,
+//               32 activation columns each, read with 16x128b loads (4
+//               weight rows x 8 activation columns per thread).
 //
 // Epilogue arithmetic (per element and block, exact up to one rounding in
 // each of two FMAs):
@@ -61,15 +60,18 @@ constexpr int KS = 32 * KBS;      // bytes of K per stage
 constexpr int STAGES = 5;
 constexpr int TBUF = 4;           // tensor-memory ring depth (x BM columns)
 constexpr int TMEM_COLS = TBUF * BM;
-constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 384;
+constexpr int EPI_WARPS = 16;
+constexpr int THREADS = 640;
 constexpr int EPI_WARP0 = 4;
-// Register split: launched with 384 x 168 = 64512 registers; the control
-// warpgroup (warps 0-3) drops to 56 and the two epilogue warpgroups rise to
-// 224: 128 x 56 + 256 x 224 = 64512.
-constexpr int CTRL_REGS = 56;
-constexpr int EPI_REGS = 224;
-static_assert(128 * CTRL_REGS + 256 * EPI_REGS <= THREADS * 168, "register split exceeds the launch allocation");
+// Register split: launched with 640 x 96 = 61440 registers (the most that
+// 640 threads can hold); the control warpgroup (warps 0-3) drops to 64 and
+// the four epilogue warpgroups rise to 104: 128 x 64 + 512 x 104 = 61440.
+constexpr int LAUNCH_REGS = 96;
+constexpr int CTRL_REGS = 64;
+constexpr int EPI_REGS = 104;
+static_assert(THREADS * LAUNCH_REGS <= 65536, "launch register budget");
+static_assert(128 * CTRL_REGS + (THREADS - 128) * EPI_REGS <= THREADS * LAUNCH_REGS,
+              "register split exceeds the launch allocation");
 
 constexpr int W_TILE = BN * KS;             // 16384
 constexpr int A_TILE = BM * KS;             // 16384
@@ -248,22 +250,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         const bool exotic = __any_sync(0xFFFFFFFFu, bad);
-        if (!exotic) {
-          // a_scale * 2^49 and W = w_scale * 2^100, both exact inside the window
+        // a_scale * 2^49 and W = w_scale * 2^100 (exact inside the window;
+        // an exotic stage keeps the scales as loaded)
+        const float fa = exotic ? 1.0f : 0x1p49f;
+        const float fw = exotic ? 1.0f : 0x1p100f;
+        __syncwarp();
+        // Rewrite both scale tiles in the order the epilogue reads them.
+        // Activation scales [kb][m], m = 32h + r + 4k  ->  [kb][h][r][k]:
+        // lane L holds m = 4L..4L+3 of every kb (h = L/8, k = L%8, r = e).
+        // Weight scales [n][kb], n = 32q + l + 8i  ->  [kb][q][l][i]: lane L
+        // holds row n = 32j + L (q = j, l = L%8, i = L/8) for all four kb.
+        float* asf = reinterpret_cast<float*>(st + OFF_AS);
+        float* wsf = reinterpret_cast<float*>(st + OFF_WS);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            float4 v = av[j];
-            v.x *= 0x1p49f;
-            v.y *= 0x1p49f;
-            v.z *= 0x1p49f;
-            v.w *= 0x1p49f;
-            as4[j * 32 + lane] = v;
-            float4 w = wv[j];
-            w.x *= 0x1p100f;
-            w.y *= 0x1p100f;
-            w.z *= 0x1p100f;
-            w.w *= 0x1p100f;
-            ws4[j * 32 + lane] = w;
+        for (int j = 0; j < 4; ++j) {
+          const float a4[4] = {av[j].x, av[j].y, av[j].z, av[j].w};
+          const float w4[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            asf[j * BM + (lane >> 3) * 32 + e * 8 + (lane & 7)] = a4[e] * fa;
+            wsf[e * BN + j * 32 + (lane & 7) * 4 + (lane >> 3)] = w4[e] * fw;
           }
         }
         if (lane == 0) ctrl->exotic[s] = exotic ? 1 : 0;
@@ -276,85 +282,46 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     setmaxnreg_inc<EPI_REGS>();
     // ---------------------------------------------------------------- epilogue
-    // Warp (quarter q, half hc) owns tensor-memory lanes 32q..32q+31 (weight
-    // rows) and columns 64hc..64hc+63 (activation rows), read with one
-    // 32x32b.x64 load per block: thread t holds weight row 32q + t and the
-    // 64 activation rows of its half.  Its weight scales for the four blocks
-    // of a stage are one 16-byte load; the activation scales, the same for the
-    // whole warp, are broadcast 16-byte loads.  The four K blocks of a stage
-    // are unrolled (buffer = barrier = kb), and the next block's tensor-memory
-    // load is in flight while the second half of the current block is
-    // rescaled.
+    // Warp (quarter q, column slice h) owns tensor-memory lanes 32q..32q+31
+    // (weight rows) and columns 32h..32h+31 (activation rows), read per block
+    // with two 16x128b.x8 loads (lanes 32q..+15 and 32q+16..+31): thread t
+    // holds weight rows 32q + t/4 + 8i (i = 0..3) and activation columns
+    // 32h + t%4 + 4k (k = 0..7).  Registers r[2k], r[2k+1] of one load are
+    // rows (t/4, t/4 + 8) at the same column: the operand pair of one packed
+    // FMA.  Per block a thread needs 4 weight scales (one 16-byte load) and
+    // 8 activation scales (two), from the tiles the prep warp rewrote.
+    // A warp hands its buffer back as soon as its loads have landed and then
+    // rescales from registers; four warps per scheduler hide each other's
+    // load latency.
     const int q = warp & 3;
-    const int hc = (warp - EPI_WARP0) >> 2;
-    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(hc * 64);
+    const int h = (warp - EPI_WARP0) >> 2;
+    const int l8 = lane >> 2;
+    const int c4 = lane & 3;
+    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 32);
     const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const uint32_t smem_base = smem_u32(smem);
-    const uint32_t ws_off = OFF_WS + (uint32_t)((q * 32 + lane) * KBS) * 4u;  // [n][kb]
-    const uint32_t as_off = OFF_AS + (uint32_t)(hc * 64) * 4u;                // + kb*BM*4 + c*4
+    const uint32_t ws_off = OFF_WS + (uint32_t)(q * 32 + l8 * 4) * 4u;  // + kb*BN*4
+    const uint32_t as_off = OFF_AS + (uint32_t)(h * 32 + c4 * 8) * 4u;  // + kb*BM*4
 
     // open the tensor-memory ring
-    if (lane == 0)
-      for (int b = 0; b < TBUF; ++b) mbar_arrive(&ctrl->tempty[b]);
+    mbar_arrive_lane0(&ctrl->tempty[0], lane);
+    mbar_arrive_lane0(&ctrl->tempty[1], lane);
+    mbar_arrive_lane0(&ctrl->tempty[2], lane);
+    mbar_arrive_lane0(&ctrl->tempty[3], lane);
 
-    float2 acc[32];  // acc[c/2] = columns (c, c+1)
-    uint32_t pa[64], pb[64];
+    float2 acc[2][8];  // acc[j][k] = rows (2j, 2j+1) of this thread's four, column k
+    uint32_t r0[16], r1[16];
 
-    // load block kb's partials (buffer kb) once its MMA has landed
-    auto tload = [&](int kb, uint32_t parity, uint32_t (&d)[64]) -> bool {
-      if (!mbar_wait(&ctrl->tfull[kb], parity, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
-      tc_fence_after();
-      tmem_ld_x64(tl + kb * BM, d);
-      return true;
-    };
-    // after the load has landed, hand the buffer back to the MMA
-    auto trelease = [&](int kb) {
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive_lane0(&ctrl->tempty[kb], lane);
-    };
-
-    // Rescale columns c0..c0+31 of the current block (W, C: this thread's
-    // weight-row constants; exotic stages use the plain convert-multiply-fma).
-    // The choice is a template parameter: a stage runs one of two fully
-    // unrolled code paths, with no branch inside the per-block loop.
-    auto rescale = [&](auto exc, uint32_t aa, int c0, float W, const uint32_t (&p)[64]) {
-      if constexpr (!decltype(exc)::value) {
-        const float C = -(W * 0x1p-130f);
-#pragma unroll
-        for (int c = c0; c < c0 + 32; c += 4) {
-          const float4 a4 = lds_f32x4(aa + (uint32_t)c * 4u);
-          float2 u0, u1;
-          u0.x = __fmaf_rn(__uint_as_float(p[c]), W, C);
-          u0.y = __fmaf_rn(__uint_as_float(p[c + 1]), W, C);
-          u1.x = __fmaf_rn(__uint_as_float(p[c + 2]), W, C);
-          u1.y = __fmaf_rn(__uint_as_float(p[c + 3]), W, C);
-          acc[c / 2] = __ffma2_rn(u0, make_float2(a4.x, a4.y), acc[c / 2]);
-          acc[c / 2 + 1] = __ffma2_rn(u1, make_float2(a4.z, a4.w), acc[c / 2 + 1]);
-        }
-      } else {
-#pragma unroll
-        for (int c = c0; c < c0 + 32; c += 4) {
-          const float4 a4 = lds_f32x4(aa + (uint32_t)c * 4u);
-          const float av[4] = {a4.x, a4.y, a4.z, a4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float u = __fmul_rn(__int2float_rn((int)p[c + e] - (int)kBias), W);
-            float& dst = (e & 1) ? acc[(c + e) / 2].y : acc[(c + e) / 2].x;
-            dst = __fmaf_rn(u, av[e], dst);
-          }
-        }
-      }
-    };
-
-    auto dump = [&](int n0, int m0, int b, const uint32_t (&p)[64]) {
+    auto dump = [&](int n0, int m0, int b) {
       if constexpr (DUMP) {
-        const int nn = n0 + q * 32 + lane;
-        if (nn < n) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int mm = m0 + hc * 64 + c;
-            if (mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)p[c] - (int)kBias;
+        for (int i = 0; i < 4; ++i) {
+          const int nn = n0 + q * 32 + l8 + 8 * i;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int mm = m0 + h * 32 + c4 + 4 * k;
+            const uint32_t v = (i < 2) ? r0[2 * k + (i & 1)] : r1[2 * k + (i & 1)];
+            if (nn < n && mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)v - (int)kBias;
           }
         }
       }
@@ -362,45 +329,73 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     // Stage sequence of this CTA: stage counter itg (tiles x K stages), ring
     // slot itg % STAGES; within a stage the four K blocks are unrolled, block
-    // kb in tensor-memory buffer kb (phase itg & 1), with the partials of
-    // even blocks in pa and of odd blocks in pb.
+    // kb in tensor-memory buffer kb (phase itg & 1).
     const int total_st = my_tiles * kstages;
     int tile = blockIdx.x, n0 = 0, m0 = 0, kst = 0;
     tile_coords(tile, n0, m0);
     uint32_t st_addr = smem_base;
-    int exotic = 0;
-    float4 wst = make_float4(0.f, 0.f, 0.f, 0.f);
     uint32_t itg = 0;
 
-    auto sub = [&](auto kbc, auto exc, uint32_t (&cur)[64], uint32_t (&nxt)[64]) -> bool {
+    // One K block: scales, partials, buffer release, rescale.  The choice of
+    // the exotic path is a template parameter, so a stage runs one of two
+    // fully unrolled code paths with no branch inside.
+    auto sub = [&](auto kbc, auto exc) -> bool {
       constexpr int kb = decltype(kbc)::value;
-      const int s = (int)(itg % STAGES);
-      const float W = (kb == 0) ? wst.x : (kb == 1) ? wst.y : (kb == 2) ? wst.z : wst.w;
-      const uint32_t aa = st_addr + as_off + (uint32_t)kb * (BM * 4u);
-      rescale(exc, aa, 0, W, cur);
-      // next block: block kb+1 of this stage, or block 0 of the next stage
-      const bool has_next = (kb < KBS - 1) || (itg + 1 < (uint32_t)total_st);
-      if (has_next) {
-        const uint32_t par = (kb < KBS - 1) ? (itg & 1u) : ((itg + 1) & 1u);
-        if (!tload((kb + 1) & (KBS - 1), par, nxt)) return false;
-      }
-      rescale(exc, aa, 32, W, cur);
-      dump(n0, m0, kst * KBS + kb, cur);
-      if (kb == KBS - 1) {
-        mbar_arrive_lane0(&ctrl->empty[s], lane);
-        if (++kst == kstages) {
-          // tile end: write BF16 out[m][n] (lanes = consecutive n); the
-          // tile origin passes through a volatile move so the store
-          // addresses are formed here only
-          int nr, mr;
-          asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + lane));
-          asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + hc * 64));
-          if (nr < n) {
+      constexpr bool EXO = decltype(exc)::value;
+      const float4 W4 = lds_f32x4(st_addr + ws_off + (uint32_t)kb * (BN * 4u));
+      const float4 A0 = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u));
+      const float4 A1 = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u) + 16u);
+      if (!mbar_wait(&ctrl->tfull[kb], itg & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
+      tc_fence_after();
+      tmem_ld_16x128b_x8(tl + kb * BM, r0);
+      tmem_ld_16x128b_x8(tl + kb * BM + (16u << 16), r1);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive_lane0(&ctrl->tempty[kb], lane);
+      const float av[8] = {A0.x, A0.y, A0.z, A0.w, A1.x, A1.y, A1.z, A1.w};
+      const float2 Wp[2] = {make_float2(W4.x, W4.y), make_float2(W4.z, W4.w)};
+      if constexpr (!EXO) {
+        const float2 Cp[2] = {make_float2(-(W4.x * 0x1p-130f), -(W4.y * 0x1p-130f)),
+                              make_float2(-(W4.z * 0x1p-130f), -(W4.w * 0x1p-130f))};
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-              const int mm = mr + c;
-              if (mm < m) out[(size_t)mm * n + nr] = __float2bfloat16_rn(acc[c / 2].x);
-              if (mm + 1 < m) out[(size_t)(mm + 1) * n + nr] = __float2bfloat16_rn(acc[c / 2].y);
+        for (int k = 0; k < 8; ++k) {
+          const float2 u0 = __ffma2_rn(f2(r0[2 * k], r0[2 * k + 1]), Wp[0], Cp[0]);
+          const float2 u1 = __ffma2_rn(f2(r1[2 * k], r1[2 * k + 1]), Wp[1], Cp[1]);
+          acc[0][k] = __ffma2_rn(u0, make_float2(av[k], av[k]), acc[0][k]);
+          acc[1][k] = __ffma2_rn(u1, make_float2(av[k], av[k]), acc[1][k]);
+        }
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const uint32_t* rr = j ? r1 : r0;
+            const float ux = __fmul_rn(__int2float_rn((int)rr[2 * k] - (int)kBias), j ? W4.z : W4.x);
+            const float uy = __fmul_rn(__int2float_rn((int)rr[2 * k + 1] - (int)kBias), j ? W4.w : W4.y);
+            acc[j][k].x = __fmaf_rn(ux, av[k], acc[j][k].x);
+            acc[j][k].y = __fmaf_rn(uy, av[k], acc[j][k].y);
+          }
+        }
+      }
+      dump(n0, m0, kst * KBS + kb);
+      if (kb == KBS - 1) {
+        mbar_arrive_lane0(&ctrl->empty[(int)(itg % STAGES)], lane);
+        if (++kst == kstages) {
+          // tile end: write BF16 out[m][n]; the tile origin passes through a
+          // volatile move so the store addresses are formed here only
+          int nr, mr;
+          asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + l8));
+          asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + h * 32 + c4));
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int nn = nr + 8 * i;
+            if (nn < n) {
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                const int mm = mr + 4 * k;
+                const float v = (i & 1) ? acc[i >> 1][k].y : acc[i >> 1][k].x;
+                if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(v);
+              }
             }
           }
           kst = 0;
@@ -408,24 +403,20 @@ __global__ void __launch_bounds__(THREADS, 1)
           tile_coords(tile, n0, m0);
         }
       }
-      if (has_next) trelease((kb + 1) & (KBS - 1));
       return true;
     };
 
     bool ok = true;
-    if (total_st > 0) {
-      ok = tload(0, 0u, pa);
-      if (ok) trelease(0);
-    }
     for (; ok && itg < (uint32_t)total_st; ++itg) {
       const int s = (int)(itg % STAGES);
       if (!mbar_wait(&ctrl->prep[s], (itg / STAGES) & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) break;
       st_addr = smem_base + (uint32_t)s * STAGE_BYTES;
-      exotic = ctrl->exotic[s];
-      wst = lds_f32x4(st_addr + ws_off);
+      const int exotic = ctrl->exotic[s];
       if (kst == 0) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.0f, 0.0f);
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[j][k] = make_float2(0.0f, 0.0f);
       }
       using K0 = std::integral_constant<int, 0>;
       using K1 = std::integral_constant<int, 1>;
@@ -433,10 +424,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       using K3 = std::integral_constant<int, 3>;
       if (!exotic) {
         const std::false_type fast;
-        ok = sub(K0{}, fast, pa, pb) && sub(K1{}, fast, pb, pa) && sub(K2{}, fast, pa, pb) && sub(K3{}, fast, pb, pa);
+        ok = sub(K0{}, fast) && sub(K1{}, fast) && sub(K2{}, fast) && sub(K3{}, fast);
       } else {
         const std::true_type slow;
-        ok = sub(K0{}, slow, pa, pb) && sub(K1{}, slow, pb, pa) && sub(K2{}, slow, pa, pb) && sub(K3{}, slow, pb, pa);
+        ok = sub(K0{}, slow) && sub(K1{}, slow) && sub(K2{}, slow) && sub(K3{}, slow);
       }
     }
   }
