@@ -203,6 +203,21 @@ def make_activations(m: int, k: int, seed: int, recipe: str):
     return _to_bf16_bits(x), info
 
 
+def make_gate_up(m: int, k: int, seed: int):
+    """Gate and up activations [M, K] (BF16 bit patterns) for the SiLU.mul
+    quantiser, g, u ~ N(0, 1), with 0.1% of the 32-groups of u scaled by 1e-6
+    so that some products form a near-zero group (the down-projection
+    activation recipe).  Returns (g_bits, u_bits, info)."""
+    rng = np.random.default_rng(2 * seed + 1)
+    g = rng.standard_normal((m, k), dtype=np.float32)
+    u = rng.standard_normal((m, k), dtype=np.float32)
+    groups = m * (k // 32)
+    cnt = max(1, groups // 1000)
+    sel = rng.choice(groups, cnt, replace=False)
+    u.reshape(groups, 32)[sel] *= np.float32(1e-6)
+    return _to_bf16_bits(g), _to_bf16_bits(u), {"recipe": "gate_up", "near_zero_groups": np.sort(sel)}
+
+
 def make_workload(name_or_wl, weight_only=False):
     wl = WORKLOADS[name_or_wl] if isinstance(name_or_wl, str) else name_or_wl
     wt = make_weight(wl.n, wl.k, wl.seed, wl.weight_outlier_rows)

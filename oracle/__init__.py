@@ -62,6 +62,9 @@ __all__ = [
     "bf16_rne",
     "proj_rows",
     "proj",
+    "exp_f32",
+    "silu_mul_bf16",
+    "requant_silu_a",
 ]
 
 GROUP = 32  # elements per int8 scale group
@@ -230,3 +233,80 @@ def proj(a_bits, w_packed, w_e4m3, scale2, k: int) -> np.ndarray:
     """The whole path from the NVFP4 weight: requant_w, then proj_rows."""
     w_i8, w_scale = requant_w(w_packed, w_e4m3, scale2, k)
     return proj_rows(a_bits, w_i8, w_scale)
+
+
+# ---------------------------------------------------------------------------
+# SiLU.mul quantiser
+#
+# The pages name a quantiser of the SiLU product (w8a8_decode/parts.rs,
+# ``W8a8Kernels::quant_silu``; the gate+up step of the grouped decode page,
+# ``moe_expert_gate_up_act_fp8_grouped_tc_w8a8``, writes "quantized
+# products") but give no arithmetic for it.  Reading taken: the product is
+# the BF16 activation the down projection would otherwise receive,
+#     x = bf16_rne(silu(g) * u),   silu(g) = g / (1 + exp(-g)),
+# every step a float32 operation rounded to nearest, and the quantiser is
+# requant_a of x.  exp is spelled out below so that a GPU implementation can
+# follow the same steps and agree bit for bit.
+# ---------------------------------------------------------------------------
+
+# float32 constants, by bit pattern
+_LOG2E = np.uint32(0x3FB8AA3B).view(np.float32)    # 1.442695
+_LN2_HI = np.uint32(0x3F317200).view(np.float32)   # 0.693145751953125 (15 significant bits)
+_LN2_LO = np.uint32(0x35BFBE8E).view(np.float32)   # ln 2 - _LN2_HI
+_EXP_COEF = [np.uint32(b).view(np.float32) for b in
+             (0x3F800000, 0x3F800000, 0x3F000000, 0x3E2AAAAB, 0x3D2AAAAB, 0x3C088889, 0x3AB60B61)]  # 1/i!
+
+
+def _pow2_f32(h: np.ndarray) -> np.ndarray:
+    """2^h as float32 for integer h in [-126, 127] (exact)."""
+    return ((h.astype(np.int64) + 127) << 23).astype(np.uint32).view(np.float32)
+
+
+def exp_f32(x) -> np.ndarray:
+    """exp in float32 by Cody-Waite range reduction and a degree-6 Taylor
+    polynomial, every operation a float32 multiply or add rounded to nearest
+    (no fused multiply-add):
+
+        n = rint_half_even(x * log2e)
+        r = (x - n * ln2_hi) - n * ln2_lo          (n * ln2_hi is exact)
+        p = 1 + r(1 + r(1/2 + r(1/6 + r(1/24 + r(1/120 + r/720)))))   (Horner)
+        exp(x) = (p * 2^h1) * 2^h2,  h1 = floor(n/2), h2 = n - h1
+
+    x > 88 gives +inf, x < -88 gives +0, NaN stays NaN."""
+    x = np.asarray(x, dtype=np.float32)
+    f32 = np.float32
+    with np.errstate(over="ignore", invalid="ignore", under="ignore"):
+        xc = np.clip(x, f32(-88.0), f32(88.0))
+        xc = np.where(np.isnan(xc), f32(0.0), xc).astype(np.float32)
+        n = np.rint((xc * _LOG2E).astype(np.float32)).astype(np.float32)
+        r = ((xc - (n * _LN2_HI).astype(np.float32)).astype(np.float32) - (n * _LN2_LO).astype(np.float32))
+        r = r.astype(np.float32)
+        p = _EXP_COEF[6]
+        for c in _EXP_COEF[5::-1]:
+            p = ((p * r).astype(np.float32) + c).astype(np.float32)
+        ni = n.astype(np.int64)
+        h1 = ni >> 1
+        h2 = ni - h1
+        y = ((p * _pow2_f32(h1)).astype(np.float32) * _pow2_f32(h2)).astype(np.float32)
+    y = np.where(x > f32(88.0), f32(np.inf), y)
+    y = np.where(x < f32(-88.0), f32(0.0), y)
+    return np.where(np.isnan(x), x, y).astype(np.float32)
+
+
+def silu_mul_bf16(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
+    """BF16 bits of silu(g) * u from BF16 g and u (bit patterns):
+    e = exp_f32(-g), s = g / (1 + e), x = s * u, each rounded to float32, then
+    bf16_rne(x)."""
+    g = bf16_bits_to_f32(np.asarray(g_bits, dtype=np.uint16))
+    u = bf16_bits_to_f32(np.asarray(u_bits, dtype=np.uint16))
+    with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
+        e = exp_f32(-g)
+        d = (np.float32(1.0) + e).astype(np.float32)
+        s = (g / d).astype(np.float32)
+        x = (s * u).astype(np.float32)
+    return bf16_rne(x)
+
+
+def requant_silu_a(g_bits: np.ndarray, u_bits: np.ndarray):
+    """The SiLU.mul quantiser: requant_a of silu_mul_bf16(g, u)."""
+    return requant_a(silu_mul_bf16(g_bits, u_bits))
