@@ -18,6 +18,9 @@ Operations (gemm_dense_int8.rs launcher page):
   rescale, F32 accumulation, BF16 output.
 * :func:`proj` -- ``int8_gemm_faith2_prefill``: the whole projection from BF16
   activations (decode kernel for M <= 16, requant_a + gemm otherwise).
+* :func:`silu_mul`, :func:`requant_silu_a`, :func:`proj_silu` -- the SiLU.mul
+  quantiser (``W8a8Kernels::quant_silu``) and the down projection from gate
+  and up activations.
 """
 from __future__ import annotations
 
@@ -40,11 +43,18 @@ __all__ = [
     "decode",
     "DECODE_MAX_M",
     "STATUS_NAMES",
+    "DEV_STATUS_DEBUG_WAIT",
+    "debug_wait_timeout",
+    "silu_mul",
+    "requant_silu_a",
+    "proj_silu_scratch_bytes",
+    "proj_silu",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsr.so")
 DECODE_MAX_M = 16
+DEV_STATUS_DEBUG_WAIT = 32  # device status bit of bsr_debug_wait_timeout
 
 STATUS_NAMES = {
     0: "BSR_OK",
@@ -73,6 +83,11 @@ SIGNATURES = [
     ("bsr_decode", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_gemm_partials", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_proj_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    ("bsr_debug_wait_timeout", ctypes.c_int, [ctypes.c_int, _P]),
+    ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
+    ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
+    ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
+    ("bsr_proj_silu", ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P]),
 ]
 
 
@@ -314,6 +329,91 @@ def decode(a, w_i8, w_scale, out=None, stream=None):
             m,
             n,
             k,
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def debug_wait_timeout(limit_ms: int, stream=None):
+    """Queue the test kernel whose one pipeline wait can never be satisfied;
+    it gives up after ``limit_ms`` and sets bit 32 of the device status word
+    (read it with :func:`device_status`)."""
+    _check(lib().bsr_debug_wait_timeout(int(limit_ms), _stream_ptr(stream)))
+
+
+def silu_mul(gate, up, x=None, stream=None):
+    """x = bf16(silu(gate) * up), all [M, K] bfloat16."""
+    torch = _torch()
+    m, k = gate.shape
+    if x is None:
+        x = _empty((m, k), torch.bfloat16, gate)
+    _check(
+        lib().bsr_silu_mul(
+            _dev(gate, torch.bfloat16, (m, k), "gate"),
+            _dev(up, torch.bfloat16, (m, k), "up"),
+            _dev(x, torch.bfloat16, (m, k), "x"),
+            m,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return x
+
+
+def requant_silu_a(gate, up, a_i8=None, a_scale_t=None, stream=None):
+    """requant_a of bf16(silu(gate) * up) -> (a_i8 [M, K], a_scale_t [K/32, ld])."""
+    torch = _torch()
+    m, k = gate.shape
+    ld = a_scale_ld(m)
+    if a_i8 is None:
+        a_i8 = _empty((m, k), torch.int8, gate)
+    if a_scale_t is None:
+        a_scale_t = _empty((k // 32, ld), torch.float32, gate)
+    _check(
+        lib().bsr_requant_silu_a(
+            _dev(gate, torch.bfloat16, (m, k), "gate"),
+            _dev(up, torch.bfloat16, (m, k), "up"),
+            _dev(a_i8, torch.int8, (m, k), "a_i8"),
+            _dev(a_scale_t, torch.float32, (k // 32, ld), "a_scale_t"),
+            m,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return a_i8, a_scale_t
+
+
+def proj_silu_scratch_bytes(m: int, k: int) -> int:
+    return lib().bsr_proj_silu_scratch_bytes(m, k)
+
+
+def proj_silu(gate, up, w_i8, w_scale, out=None, scratch=None, stream=None):
+    """out [M, N] bfloat16 = proj(bf16(silu(gate) * up), W)."""
+    torch = _torch()
+    m, k = gate.shape
+    n = w_i8.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, gate)
+    need = proj_silu_scratch_bytes(m, k)
+    if scratch is None and need:
+        scratch = _empty((need,), torch.uint8, gate)
+    if scratch is not None and not scratch.is_cuda:
+        raise ValueError("scratch must be a CUDA tensor")
+    sp = ctypes.c_void_p(scratch.data_ptr()) if scratch is not None else ctypes.c_void_p(0)
+    sb = scratch.numel() * scratch.element_size() if scratch is not None else 0
+    _check(
+        lib().bsr_proj_silu(
+            _dev(gate, torch.bfloat16, (m, k), "gate"),
+            _dev(up, torch.bfloat16, (m, k), "up"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            sp,
+            sb,
             _stream_ptr(stream),
         )
     )

@@ -245,6 +245,15 @@ size_t bsr_proj_scratch_bytes(int64_t m, int64_t k) {
   return align256((size_t)m * (size_t)k) + (size_t)(k / 32) * (size_t)a_scale_ld(m) * 4;
 }
 
+bsr_status bsr_debug_wait_timeout(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return fail(BSR_EINVAL, "bsr_debug_wait_timeout: limit_ms %d not in [1, 2000]", limit_ms);
+  DevInfo d;
+  bsr_status st = device_info(d);
+  if (st != BSR_OK) return st;
+  return cuda_status(bsr::launch_debug_wait(d.status, (unsigned long long)limit_ms * 1000000ull, as_stream(stream)),
+                     "debug wait launch");
+}
+
 bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
                       int64_t n, int64_t k, void* stream) {
   bsr_status st = check_dims(m, n, k, true, true);
@@ -268,6 +277,65 @@ bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale,
   int8_t* a_i8 = static_cast<int8_t*>(scratch);
   float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
   if ((st = bsr_requant_a(a, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
+  return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
+}
+
+bsr_status bsr_silu_mul(const uint16_t* gate, const uint16_t* up, uint16_t* x, int64_t m, int64_t k, void* stream) {
+  bsr_status st = check_dims(m, 0, k, true, false);
+  if (st != BSR_OK) return st;
+  if (m == 0) return ok();
+  if (!gate || !up || !x) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(x))
+    return fail(BSR_EALIGN, "bsr_silu_mul: pointers must be 16-byte aligned");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  return cuda_status(bsr::launch_silu_mul(gate, up, x, (int)m, (int)k, as_stream(stream), d.num_sms),
+                     "silu_mul launch");
+}
+
+bsr_status bsr_requant_silu_a(const uint16_t* gate, const uint16_t* up, int8_t* a_i8, float* a_scale_t, int64_t m,
+                              int64_t k, void* stream) {
+  bsr_status st = check_dims(m, 0, k, true, false);
+  if (st != BSR_OK) return st;
+  if (m == 0) return ok();
+  if (!gate || !up || !a_i8 || !a_scale_t) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(a_i8) || !aligned16(a_scale_t))
+    return fail(BSR_EALIGN, "bsr_requant_silu_a: pointers must be 16-byte aligned");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  return cuda_status(bsr::launch_requant_silu_a(gate, up, a_i8, a_scale_t, (int)m, (int)k, (int)a_scale_ld(m),
+                                                as_stream(stream), d.num_sms),
+                     "requant_silu_a launch");
+}
+
+size_t bsr_proj_silu_scratch_bytes(int64_t m, int64_t k) {
+  if (m <= 0 || k <= 0 || k % 32 != 0) return 0;
+  if (m <= BSR_DECODE_MAX_M || k % 128 != 0) return align256((size_t)m * (size_t)k * 2);  // BF16 product
+  return bsr_proj_scratch_bytes(m, k);
+}
+
+bsr_status bsr_proj_silu(const uint16_t* gate, const uint16_t* up, const int8_t* w_i8, const float* w_scale,
+                         uint16_t* out, int64_t m, int64_t n, int64_t k, void* scratch, size_t scratch_bytes,
+                         void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if ((st = check_proj_args(gate, w_i8, w_scale, out)) != BSR_OK) return st;
+  if (!up) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(up)) return fail(BSR_EALIGN, "bsr_proj_silu: pointers must be 16-byte aligned");
+  const size_t need = bsr_proj_silu_scratch_bytes(m, k);
+  if (!scratch || scratch_bytes < need)
+    return fail(BSR_ESCRATCH, "scratch of %zu bytes needed, %zu given", need, scratch ? scratch_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
+  if (m <= BSR_DECODE_MAX_M || k % 128 != 0) {
+    // decode route: the BF16 product into scratch, then the decode kernel
+    uint16_t* x = static_cast<uint16_t*>(scratch);
+    if ((st = bsr_silu_mul(gate, up, x, m, k, stream)) != BSR_OK) return st;
+    return decode_impl(x, w_i8, w_scale, out, m, n, k, stream);
+  }
+  int8_t* a_i8 = static_cast<int8_t*>(scratch);
+  float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
+  if ((st = bsr_requant_silu_a(gate, up, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
   return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
 }
 

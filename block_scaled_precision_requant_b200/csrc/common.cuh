@@ -22,6 +22,7 @@ enum : int {
   DEV_ERR_TIMEOUT_EPI = 4,
   DEV_ERR_TIMEOUT_PREP = 8,
   DEV_ERR_TIMEOUT_DECODE = 16,
+  DEV_ERR_TIMEOUT_DEBUG = 32,  // the test entry's deliberate wait
 };
 
 // 1 s of waiting on one barrier is far beyond any legal schedule here.
@@ -111,7 +112,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // raises `abort_flag` plus a bit in g_dev_status) when the wait exceeds the
 // time limit or another role of the CTA has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int* status,
-                                          int err_bit) {
+                                          int err_bit, unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
   uint32_t spins = 0;
@@ -119,7 +120,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 15u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicOr(status, err_bit);
         return false;

@@ -26,4 +26,15 @@ size_t gemm_smem_bytes();
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
                         cudaStream_t stream, int num_sms);
 
+// SiLU.mul: x = bf16(silu(g) * u) (x, g, u [M, K] BF16), and the fused
+// quantiser requant_a(bf16(silu(g) * u)) into the requant_a layout.
+cudaError_t launch_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* x, int m, int k, cudaStream_t stream,
+                            int num_sms);
+cudaError_t launch_requant_silu_a(const uint16_t* g, const uint16_t* u, int8_t* a_i8, float* a_scale_t, int m, int k,
+                                  int ld, cudaStream_t stream, int num_sms);
+
+// Test entry: one CTA waits on an mbarrier nothing arrives on, through the
+// bounded wait of the pipelined kernels, for at most limit_ns.
+cudaError_t launch_debug_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);
+
 }  // namespace bsr

@@ -135,33 +135,6 @@ __global__ void __launch_bounds__(256) requant_w_kernel(const uint4* __restrict_
 // one 32-byte segment of the block-major scale array.
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&x)[8]) {
-  x[0] = __uint_as_float(v.x << 16);
-  x[1] = __uint_as_float(v.x & 0xFFFF0000u);
-  x[2] = __uint_as_float(v.y << 16);
-  x[3] = __uint_as_float(v.y & 0xFFFF0000u);
-  x[4] = __uint_as_float(v.z << 16);
-  x[5] = __uint_as_float(v.z & 0xFFFF0000u);
-  x[6] = __uint_as_float(v.w << 16);
-  x[7] = __uint_as_float(v.w & 0xFFFF0000u);
-}
-
-// Quantise 8 consecutive values of a group whose 4 lanes are adjacent
-// (lane & ~3 .. lane | 3).  Returns the 8 codes packed, and the group scale.
-__device__ __forceinline__ uint2 quant8_quad(const float (&x)[8], float& scale_out) {
-  float amax = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(x[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
-  const GroupScale g = group_scale(amax);
-  scale_out = g.scale;
-  int q[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) q[i] = (g.scale == 0.0f) ? 0 : quant_code(x[i], g);
-  return make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
-}
-
 __global__ void __launch_bounds__(256) requant_a_kernel(const uint4* __restrict__ a, uint2* __restrict__ a_i8,
                                                         float* __restrict__ a_scale_t, int m, int k, int ld) {
   const int lane = threadIdx.x & 31;

@@ -81,9 +81,10 @@ int bsr_abi_version(void);
 const char* bsr_last_error(void);
 
 /* Synchronises the current device, returns and clears the device status
- * word: 0 if no kernel aborted a wait since the last call, else a bit set
- * (1 TMA producer, 2 MMA issuer, 4 epilogue, 8 scale preparation timed out).
- * Returns -1 if the device could not be queried. */
+ * word: 0 if no kernel aborted a wait since the last call, else the OR of
+ * bits naming the waits that ran out (GEMM: 1 TMA producer, 2 MMA issuer,
+ * 4 epilogue, 8 scale preparation; 16 decode kernel; 32 the test entry
+ * bsr_debug_wait_timeout).  Returns -1 if the device could not be queried. */
 int bsr_device_status(void);
 
 /*
@@ -170,6 +171,43 @@ bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scal
 bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
                              uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream);
 
+/*
+ * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
+ * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:
+ *   x = bf16_rne(silu(g) * u),  silu(g) = g / (1 + exp(-g)),
+ * each step a float32 operation rounded to nearest, exp by fixed steps
+ * (Cody-Waite reduction, degree-6 Taylor polynomial; within 3 ulp of exp on
+ * [-88, 88], +inf above 88, +0 below -88).  Inputs gate, up: [M, K] BF16,
+ * finite.  Requirements and errors as bsr_requant_a.
+ */
+
+/* x [M, K] BF16 out: the product itself (the unfused activation). */
+bsr_status bsr_silu_mul(const uint16_t* gate, const uint16_t* up, uint16_t* x, int64_t m, int64_t k, void* stream);
+
+/* requant_a of the product without writing it: a_i8 [M, K] int8 and
+ * a_scale_t [K/32, bsr_a_scale_ld(M)] float out, bit-identical to
+ * bsr_silu_mul followed by bsr_requant_a. */
+bsr_status bsr_requant_silu_a(const uint16_t* gate, const uint16_t* up, int8_t* a_i8, float* a_scale_t, int64_t m,
+                              int64_t k, void* stream);
+
+/* Scratch bytes bsr_proj_silu needs: bsr_proj_scratch_bytes(M, K) on the
+ * tensor-core route (M > BSR_DECODE_MAX_M and K % 128 == 0), else the BF16
+ * product, 2*M*K rounded up to 256 (0 for invalid sizes). */
+size_t bsr_proj_silu_scratch_bytes(int64_t m, int64_t k);
+
+/*
+ * bsr_proj_silu -- the down projection from gate and up:
+ *   out = proj(bf16(silu(gate) * up), W).
+ * M > BSR_DECODE_MAX_M and K % 128 == 0: bsr_requant_silu_a into scratch,
+ * then the tensor-core GEMM (the BF16 product is never written).  Otherwise:
+ * bsr_silu_mul into scratch, then the decode kernel.  Same results as
+ * bsr_silu_mul followed by bsr_proj.  Scratch (caller-owned, device,
+ * 256-byte aligned) of at least bsr_proj_silu_scratch_bytes(M, K).
+ */
+bsr_status bsr_proj_silu(const uint16_t* gate, const uint16_t* up, const int8_t* w_i8, const float* w_scale,
+                         uint16_t* out, int64_t m, int64_t n, int64_t k, void* scratch, size_t scratch_bytes,
+                         void* stream);
+
 /* Size of the device array bsr_proj_noalloc uses as its scratch: 16 MiB,
  * enough for M*K + (K/32)*round_up(M,4)*4 <= 16 MiB (e.g. M=2048, K=4096 or
  * M=3584, K=4096; not M=4095, K=8192). */
@@ -193,6 +231,17 @@ bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const i
  */
 bsr_status bsr_proj_noalloc(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
                             int64_t n, int64_t k, void* stream);
+
+/*
+ * bsr_debug_wait_timeout -- test entry for the failure path; no counterpart
+ * on the launcher pages.  Launches one CTA that waits on an mbarrier nothing
+ * ever arrives on, through the same bounded wait the pipelined kernels use,
+ * with a limit of limit_ms milliseconds (1..2000, else BSR_EINVAL).  When the
+ * limit runs out the kernel sets bit 32 of the device status word and
+ * returns; no fault, no trap, and the device stays usable.  Returns once the
+ * kernel is queued; bsr_device_status() then waits for it and reports 32.
+ */
+bsr_status bsr_debug_wait_timeout(int limit_ms, void* stream);
 
 #ifdef __cplusplus
 }

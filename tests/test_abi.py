@@ -72,6 +72,12 @@ def test_invalid_and_alignment_errors(L):
                                None) == 1
 
 
+def test_debug_wait_limit_checked_before_launch(L):
+    assert L.bsr_debug_wait_timeout(0, None) == 1
+    assert L.bsr_debug_wait_timeout(2001, None) == 1
+    assert "limit_ms" in bsr.last_error()
+
+
 def test_scratch_errors(L):
     m, k = 64, 256
     need = L.bsr_proj_scratch_bytes(m, k)
