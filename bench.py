@@ -44,8 +44,11 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 L2_FLUSH_BYTES = 256 << 20
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
 INT8_PER_BF16 = 2.0  # nominal dense int8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+# The exact per-block rescale costs 2 FP32 FMAs per output element and 32-wide
+# K block (= 64 int8 ops); the FP32 pipe retires 128 FMAs per clock per SM.
+OPS_PER_SM_CLOCK_FMA_BOUND = 64 * 128 / 2
 
 
 def parse_args(argv=None):
@@ -259,6 +262,12 @@ def prefill_ops(m, n, k):
     return 2 * m * n * k
 
 
+def fma_bound_tops(num_sms, sm_mhz):
+    """int8 ops/s of the GEMM when the FP32 pipe does nothing but the exact
+    rescale (2 FMAs per element and 32-block), in TOPS."""
+    return OPS_PER_SM_CLOCK_FMA_BOUND * num_sms * sm_mhz * 1e6 / 1e12
+
+
 class Gpu:
     """Device state of one workload: requantised weight resident in HBM."""
 
@@ -275,6 +284,7 @@ class Gpu:
         self.host = d
         m, n, k = self.wl.shape
         self.dev = device
+        self.num_sms = torch.cuda.get_device_properties(device).multi_processor_count
         wp = torch.from_numpy(d["w_packed"]).to(device)
         we = torch.from_numpy(d["w_e4m3"]).to(device)
         self.w_i8, self.w_s = bsr.requant_w(wp, we, float(d["scale2"]))
@@ -313,15 +323,18 @@ class Gpu:
         copies = max(2, -(-3 * l2 // wbytes))
         ws = [(self.w_i8.clone(), self.w_s.clone()) for _ in range(copies)]
         bsr = self.bsr
+        # the weight copies are written before the capture and never inside
+        # it, so every step may start its weight stream before the previous
+        # step ends (the static-weight decode option)
         for i in range(max(warmup, 1)):  # eager warm-up also fills the launch caches
             w, s = ws[i % copies]
-            bsr.proj(self.a, w, s, self.out)
+            bsr.decode(self.a, w, s, self.out, static_weight=True)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for i in range(steps):
                 w, s = ws[i % copies]
-                bsr.proj(self.a, w, s, self.out)
+                bsr.decode(self.a, w, s, self.out, static_weight=True)
         g.replay()  # warm replay
         torch.cuda.synchronize()
         dist_barrier()
@@ -481,20 +494,53 @@ def prefill_extra(name, device, steps, warmup, peaks):
     t_rw = mean_ms(g.timed_requant_w_only(steps, warmup))
     g.check_status()
     int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
+    fma_peak = fma_bound_tops(g.num_sms, peaks["sm_max_mhz"])
     res = {
         "shape": [m, n, k],
         "tops_incl_requant": ops / t_step / 1e9,
         "gemm_tops": ops / t_gemm / 1e9,
         "gemm_frac_of_int8_peak": ops / t_gemm / 1e9 / int8_peak,
+        "gemm_frac_of_fma_bound": ops / t_gemm / 1e9 / fma_peak,
         "requant_a_gbs": m * k * 3.125 / t_ra / 1e6,
         "requant_w_gbs": n * k * 1.6875 / t_rw / 1e6,
         "ms": {"step": t_step, "gemm": t_gemm, "requant_a": t_ra, "requant_w": t_rw},
     }
+    if g.wl.act == "silu_mul":
+        res["silu"] = silu_extra(g, steps, warmup)
     del g
     import torch
 
     torch.cuda.empty_cache()
     return res
+
+
+def silu_extra(g, steps, warmup):
+    """The down projection from gate/up activations: the fused SiLU.mul
+    quantiser + GEMM against the unfused SiLU.mul + requant_a + GEMM."""
+    torch, bsr = g.torch, g.bsr
+    from block_scaled_precision_requant_b200 import synth
+
+    m, n, k = g.wl.shape
+    gb, ub, _ = synth.make_gate_up(m, k, g.wl.seed)
+    gate = torch.from_numpy(gb.view(np.int16)).view(torch.bfloat16).to(g.dev)
+    up = torch.from_numpy(ub.view(np.int16)).view(torch.bfloat16).to(g.dev)
+    del gb, ub
+    x = torch.empty((m, k), dtype=torch.bfloat16, device=g.dev)
+    scratch = torch.empty((bsr.proj_silu_scratch_bytes(m, k),), dtype=torch.uint8, device=g.dev)
+    t_fused = mean_ms(g.timed(lambda: bsr.proj_silu(gate, up, g.w_i8, g.w_s, g.out, scratch), steps, warmup))
+    t_quant = mean_ms(g.timed(lambda: bsr.requant_silu_a(gate, up, g.a_i8, g.a_st), steps, warmup))
+    t_mul = mean_ms(g.timed(lambda: bsr.silu_mul(gate, up, x), steps, warmup))
+    t_unfused = mean_ms(g.timed(lambda: (bsr.silu_mul(gate, up, x), bsr.proj(x, g.w_i8, g.w_s, g.out, g.scratch)),
+                                steps, warmup))
+    g.check_status()
+    ops = prefill_ops(m, n, k)
+    return {
+        "tops_fused": ops / t_fused / 1e9,
+        "tops_unfused": ops / t_unfused / 1e9,
+        "requant_silu_a_gbs": m * k * 5.125 / t_quant / 1e6,
+        "silu_mul_gbs": m * k * 6 / t_mul / 1e6,
+        "ms": {"proj_silu": t_fused, "silu_mul_then_proj": t_unfused, "requant_silu_a": t_quant, "silu_mul": t_mul},
+    }
 
 
 def gpu_main(args):
@@ -538,11 +584,18 @@ def gpu_main(args):
         rl = roofline("hbm", decode_bytes(m, n, k) / (ms_kernel / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s",
                       stored_traffic(kernel, wl.name))
     else:
-        rl = roofline("tensor", prefill_ops(m, n, k) / (ms_kernel / 1e3) / 1e12,
-                      peaks["bf16_tflops"] * INT8_PER_BF16, "TOPS", stored_traffic(kernel, wl.name))
+        # the GEMM is bound by the FP32 pipe (the exact rescale), not by the
+        # tensor pipe: report against that bound, and the tensor peak beside it
+        achieved = prefill_ops(m, n, k) / (ms_kernel / 1e3) / 1e12
+        rl = roofline("alu", achieved, fma_bound_tops(props.multi_processor_count, peaks["sm_max_mhz"]), "TOPS",
+                      stored_traffic(kernel, wl.name))
+        rl["tensor_peak"] = peaks["bf16_tflops"] * INT8_PER_BF16
+        rl["tensor_frac"] = achieved / rl["tensor_peak"]
     rl["kernel"] = kernel
     rl["peak_source"] = (f"{peak_src} (HBM copy)" if decode else
-                         f"{peak_src} bf16 cuBLAS burst x {INT8_PER_BF16:g} (nominal int8/bf16 ratio)")
+                         f"2 FP32 FMAs per element and 32-block at 128 FMA/clk/SM x {props.multi_processor_count} SMs "
+                         f"x {peaks['sm_max_mhz']:g} MHz; tensor_peak: {peak_src} bf16 cuBLAS burst x "
+                         f"{INT8_PER_BF16:g} (nominal int8/bf16 ratio)")
 
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

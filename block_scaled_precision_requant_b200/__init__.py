@@ -42,6 +42,7 @@ __all__ = [
     "proj",
     "decode",
     "DECODE_MAX_M",
+    "DECODE_STATIC_WEIGHT",
     "STATUS_NAMES",
     "DEV_STATUS_DEBUG_WAIT",
     "debug_wait_timeout",
@@ -55,6 +56,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbsr.so")
 DECODE_MAX_M = 16
 DEV_STATUS_DEBUG_WAIT = 32  # device status bit of bsr_debug_wait_timeout
+DECODE_STATIC_WEIGHT = 1  # bsr_decode_ex flag: nothing ahead on the stream writes the weight
 
 STATUS_NAMES = {
     0: "BSR_OK",
@@ -84,6 +86,7 @@ SIGNATURES = [
     ("bsr_gemm_partials", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_proj_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_debug_wait_timeout", ctypes.c_int, [ctypes.c_int, _P]),
+    ("bsr_decode_ex", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
@@ -313,15 +316,20 @@ def proj(a, w_i8, w_scale, out=None, scratch=None, stream=None):
     return out
 
 
-def decode(a, w_i8, w_scale, out=None, stream=None):
-    """The decode kernel for any M (activation requantisation fused, CUDA cores)."""
+def decode(a, w_i8, w_scale, out=None, stream=None, static_weight=False):
+    """The decode kernel for any M (activation requantisation fused, CUDA cores).
+
+    ``static_weight=True`` promises that no kernel in flight or queued ahead
+    on the stream writes ``w_i8``/``w_scale`` (a decode loop over a resident
+    weight); the kernel then starts its weight copies before waiting for the
+    previous kernel."""
     torch = _torch()
     m, k = a.shape
     n = w_i8.shape[0]
     if out is None:
         out = _empty((m, n), torch.bfloat16, a)
     _check(
-        lib().bsr_decode(
+        lib().bsr_decode_ex(
             _dev(a, torch.bfloat16, (m, k), "a"),
             _dev(w_i8, torch.int8, (n, k), "w_i8"),
             _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
@@ -329,6 +337,7 @@ def decode(a, w_i8, w_scale, out=None, stream=None):
             m,
             n,
             k,
+            DECODE_STATIC_WEIGHT if static_weight else 0,
             _stream_ptr(stream),
         )
     )

@@ -153,14 +153,14 @@ bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w
 }
 
 bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
-                       int64_t n, int64_t k, void* stream) {
+                       int64_t n, int64_t k, void* stream, int static_weight = 0) {
   DevInfo d;
   bsr_status st;
   if ((st = device_info(d)) != BSR_OK) return st;
   const int mr = bsr::decode_rows_per_cta((int)m, (int)k, d.smem_optin);
   if (mr == 0) return fail(BSR_ESHAPE, "K=%lld too large for the decode kernel's shared memory", (long long)k);
-  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, d.status, d.smem_optin,
-                                        as_stream(stream), d.num_sms),
+  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, static_weight, d.status,
+                                        d.smem_optin, as_stream(stream), d.num_sms),
                      "decode launch");
 }
 
@@ -261,6 +261,16 @@ bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scal
   if (m == 0 || n == 0) return ok();
   if ((st = check_proj_args(a, w_i8, w_scale, out)) != BSR_OK) return st;
   return decode_impl(a, w_i8, w_scale, out, m, n, k, stream);
+}
+
+bsr_status bsr_decode_ex(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                         int64_t n, int64_t k, unsigned flags, void* stream) {
+  if (flags & ~(unsigned)BSR_DECODE_STATIC_WEIGHT) return fail(BSR_EINVAL, "bsr_decode_ex: unknown flags 0x%x", flags);
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if ((st = check_proj_args(a, w_i8, w_scale, out)) != BSR_OK) return st;
+  return decode_impl(a, w_i8, w_scale, out, m, n, k, stream, (flags & BSR_DECODE_STATIC_WEIGHT) ? 1 : 0);
 }
 
 bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m, int64_t n,

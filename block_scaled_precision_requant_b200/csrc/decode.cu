@@ -81,7 +81,8 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int mr, int k, int nwar
 template <int MR>
 __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
     decode_kernel(const uint16_t* __restrict__ a, const int8_t* __restrict__ w_i8, const float* __restrict__ w_scale,
-                  __nv_bfloat16* __restrict__ out, int m, int n, int k, int scale_bulk, int* __restrict__ status) {
+                  __nv_bfloat16* __restrict__ out, int m, int n, int k, int scale_bulk, int static_weight,
+                  int* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int nb = k >> 5;
   const int warp = threadIdx.x >> 5;
@@ -99,13 +100,6 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
   const int rows = min(MR, m - m0);
   int row = blockIdx.x * nwarps + warp;
   const int row_step = gridDim.x * nwarps;
-
-  // Launched with programmatic stream serialisation: the grid may be
-  // scheduled while the previous kernel on the stream drains.  Wait for that
-  // kernel to complete (and its writes to be visible) before the first
-  // global read, and let the next kernel be scheduled early in turn.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (threadIdx.x == 0) *abort_flag = 0;
   if (lane == 0) {
@@ -143,8 +137,18 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
         v = __ldg(reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * k + (size_t)b * 32 + sub * 8));
       return v;
     };
+    // Launched with programmatic stream serialisation: the grid may be
+    // scheduled while the previous kernel on the stream drains.  Wait for
+    // that kernel to complete (and its writes to be visible) before reading
+    // what it may have written, and let the next kernel be scheduled early in
+    // turn.  With static_weight the caller guarantees that no kernel ahead
+    // on the stream writes the weight, so the first row's copies go out
+    // before the wait and overlap the previous kernel's tail.
+    if (static_weight) issue_row(row);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     uint4 av = load_act(warp * 8);
-    issue_row(row);
+    if (!static_weight) issue_row(row);
     for (int g0 = warp * 8; g0 < groups; g0 += nwarps * 8) {
       const int g = g0 + (lane >> 2);
       const int r = g / nb;
@@ -243,7 +247,8 @@ int decode_rows_per_cta(int m, int k, size_t smem_limit) {
 
 template <int MR>
 static cudaError_t launch_decode_t(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m,
-                                   int n, int k, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
+                                   int n, int k, int static_weight, int* status, size_t smem_limit,
+                                   cudaStream_t stream, int num_sms) {
   auto kern = decode_kernel<MR>;
   const bool sb = decode_scale_bulk(k);
   // Warps (= weight rows in flight) per CTA: spread the rows over all SMs,
@@ -280,19 +285,21 @@ static cudaError_t launch_decode_t(const uint16_t* a, const int8_t* w_i8, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
-  e = cudaLaunchKernelEx(&cfg, kern, a, w_i8, w_scale, o, m, n, k, sb ? 1 : 0, status);
+  e = cudaLaunchKernelEx(&cfg, kern, a, w_i8, w_scale, o, m, n, k, sb ? 1 : 0, static_weight ? 1 : 0, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
-                          int k, int mr, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
+                          int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                          int num_sms) {
+  const int sw = static_weight;
   switch (mr) {
-    case 1: return launch_decode_t<1>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
-    case 2: return launch_decode_t<2>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
-    case 4: return launch_decode_t<4>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
-    case 8: return launch_decode_t<8>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
-    case 16: return launch_decode_t<16>(a, w_i8, w_scale, out, m, n, k, status, smem_limit, stream, num_sms);
+    case 1: return launch_decode_t<1>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
+    case 2: return launch_decode_t<2>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
+    case 4: return launch_decode_t<4>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
+    case 8: return launch_decode_t<8>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
+    case 16: return launch_decode_t<16>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -21,7 +21,8 @@ cudaError_t launch_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, 
                              cudaStream_t stream, int num_sms);
 int decode_rows_per_cta(int m, int k, size_t smem_limit);
 cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
-                          int k, int mr, int* status, size_t smem_limit, cudaStream_t stream, int num_sms);
+                          int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                          int num_sms);
 size_t gemm_smem_bytes();
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
                         cudaStream_t stream, int num_sms);

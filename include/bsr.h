@@ -171,6 +171,18 @@ bsr_status bsr_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scal
 bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
                              uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream);
 
+/* bsr_decode_ex flag: no kernel that writes w_i8 or w_scale is in flight or
+ * queued ahead of this call on the stream (e.g. a decode loop over a
+ * resident weight).  The kernel then issues its first weight copies before
+ * waiting for the previous kernel on the stream, so they overlap that
+ * kernel's tail.  Activations are still read only after that wait. */
+#define BSR_DECODE_STATIC_WEIGHT 1u
+
+/* bsr_decode with flags (0 or BSR_DECODE_STATIC_WEIGHT; other bits:
+ * BSR_EINVAL).  Same arguments, results and errors as bsr_decode. */
+bsr_status bsr_decode_ex(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                         int64_t n, int64_t k, unsigned flags, void* stream);
+
 /*
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
  * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:

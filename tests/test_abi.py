@@ -78,6 +78,11 @@ def test_debug_wait_limit_checked_before_launch(L):
     assert "limit_ms" in bsr.last_error()
 
 
+def test_decode_ex_rejects_unknown_flags(L):
+    assert L.bsr_decode_ex(_fake(256), _fake(256), _fake(256), _fake(256), 1, 8, 64, 2, None) == 1
+    assert "flags" in bsr.last_error()
+
+
 def test_scratch_errors(L):
     m, k = 64, 256
     need = L.bsr_proj_scratch_bytes(m, k)
