@@ -101,6 +101,8 @@ __device__ __forceinline__ uint2 map_word(uint32_t w, const CodeTable& t) {
   return make_uint2((p0 & ~m0) | (n0 & m0), (p1 & ~m1) | (n1 & m1));
 }
 
+constexpr int kUnroll = 4;  // requant_a: tasks per warp and pass, loads first
+
 __global__ void __launch_bounds__(256) requant_w_kernel(const uint4* __restrict__ w_packed,
                                                         const uint16_t* __restrict__ w_e4m3, float scale2,
                                                         uint4* __restrict__ w_i8, float* __restrict__ w_scale,
@@ -143,21 +145,32 @@ __global__ void __launch_bounds__(256) requant_a_kernel(const uint4* __restrict_
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
   const int sub = lane & 3;
-  for (long long t = warp0; t < tasks; t += nwarps) {
-    const int r8 = (int)(t / nb);
-    const int b = (int)(t - (long long)r8 * nb);
-    const int row = r8 * 8 + (lane >> 2);
-    const bool valid = row < m;  // uniform per group of 4 lanes
-    const long long e = (long long)(valid ? row : 0) * k + (long long)b * 32 + sub * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (valid) v = __ldg(a + (e >> 3));
-    float x[8];
-    bf16x8_to_f32(v, x);
-    float s;
-    const uint2 c = quant8_quad(x, s);
-    if (valid) {
-      a_i8[e >> 3] = c;
-      if (sub == 0) a_scale_t[(long long)b * ld + row] = s;
+  // Four tasks per warp and pass, their loads issued before any arithmetic.
+  for (long long t0 = warp0; t0 < tasks; t0 += kUnroll * nwarps) {
+    uint4 v[kUnroll];
+    long long e[kUnroll];
+    int row[kUnroll], blk[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long t = t0 + u * nwarps;
+      const int r8 = (int)(t / nb);
+      blk[u] = (int)(t - (long long)r8 * nb);
+      row[u] = r8 * 8 + (lane >> 2);
+      const bool valid = t < tasks && row[u] < m;  // uniform per group of 4 lanes
+      e[u] = valid ? (long long)row[u] * k + (long long)blk[u] * 32 + sub * 8 : -1;
+      v[u] = valid ? __ldg(a + (e[u] >> 3)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (t0 + u * nwarps >= tasks) break;  // uniform per warp
+      float x[8];
+      bf16x8_to_f32(v[u], x);
+      float s;
+      const uint2 c = quant8_quad(x, s);
+      if (e[u] >= 0) {
+        a_i8[e[u] >> 3] = c;
+        if (sub == 0) a_scale_t[(long long)blk[u] * ld + row[u]] = s;
+      }
     }
   }
 }
