@@ -46,6 +46,9 @@ __all__ = [
     "STATUS_NAMES",
     "DEV_STATUS_DEBUG_WAIT",
     "debug_wait_timeout",
+    "MAX_SEGMENTS",
+    "decode_stacked",
+    "proj_stacked",
     "silu_mul",
     "requant_silu_a",
     "proj_silu_scratch_bytes",
@@ -57,6 +60,7 @@ LIB_PATH = os.path.join(_PKG, "libbsr.so")
 DECODE_MAX_M = 16
 DEV_STATUS_DEBUG_WAIT = 32  # device status bit of bsr_debug_wait_timeout
 DECODE_STATIC_WEIGHT = 1  # bsr_decode_ex flag: nothing ahead on the stream writes the weight
+MAX_SEGMENTS = 8  # BSR_MAX_SEGMENTS: segments of a stacked weight
 
 STATUS_NAMES = {
     0: "BSR_OK",
@@ -87,6 +91,8 @@ SIGNATURES = [
     ("bsr_proj_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_debug_wait_timeout", ctypes.c_int, [ctypes.c_int, _P]),
     ("bsr_decode_ex", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
+    ("bsr_decode_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, ctypes.c_uint, _P]),
+    ("bsr_proj_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
@@ -424,6 +430,66 @@ def proj_silu(gate, up, w_i8, w_scale, out=None, scratch=None, stream=None):
             sp,
             sb,
             _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def _segments(segments, k):
+    """Host arrays (device pointers and row counts) for a stacked weight given
+    as a list of (w_i8 [n_s, K], w_scale [n_s, K/32]) pairs."""
+    torch = _torch()
+    num = len(segments)
+    if not 1 <= num <= MAX_SEGMENTS:
+        raise ValueError(f"1..{MAX_SEGMENTS} segments, got {num}")
+    w_arr = (ctypes.c_void_p * num)()
+    s_arr = (ctypes.c_void_p * num)()
+    n_arr = (ctypes.c_int64 * num)()
+    for i, (w, ws) in enumerate(segments):
+        n_s = w.shape[0]
+        w_arr[i] = _dev(w, torch.int8, (n_s, k), f"w_i8[{i}]")
+        s_arr[i] = _dev(ws, torch.float32, (n_s, k // 32), f"w_scale[{i}]")
+        n_arr[i] = n_s
+    return w_arr, s_arr, n_arr, num, sum(int(w.shape[0]) for w, _ in segments)
+
+
+def decode_stacked(a, segments, out=None, stream=None, static_weight=False):
+    """One decode launch over a stacked weight: out [M, sum n_s], segment s in
+    its own column slice (segments: list of (w_i8, w_scale))."""
+    torch = _torch()
+    m, k = a.shape
+    w_arr, s_arr, n_arr, num, n = _segments(segments, k)
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    _check(
+        lib().bsr_decode_stacked(
+            _dev(a, torch.bfloat16, (m, k), "a"), ctypes.cast(w_arr, ctypes.c_void_p),
+            ctypes.cast(s_arr, ctypes.c_void_p), ctypes.cast(n_arr, ctypes.c_void_p), num,
+            _dev(out, torch.bfloat16, (m, n), "out"), m, k,
+            DECODE_STATIC_WEIGHT if static_weight else 0, _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def proj_stacked(a, segments, out=None, scratch=None, stream=None):
+    """bsr_proj over a stacked weight (decode launch for M <= 16, else
+    requant_a once and one GEMM per segment)."""
+    torch = _torch()
+    m, k = a.shape
+    w_arr, s_arr, n_arr, num, n = _segments(segments, k)
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    need = proj_scratch_bytes(m, k)
+    if scratch is None and need:
+        scratch = _empty((need,), torch.uint8, a)
+    sp = ctypes.c_void_p(scratch.data_ptr()) if scratch is not None else ctypes.c_void_p(0)
+    sb = scratch.numel() * scratch.element_size() if scratch is not None else 0
+    _check(
+        lib().bsr_proj_stacked(
+            _dev(a, torch.bfloat16, (m, k), "a"), ctypes.cast(w_arr, ctypes.c_void_p),
+            ctypes.cast(s_arr, ctypes.c_void_p), ctypes.cast(n_arr, ctypes.c_void_p), num,
+            _dev(out, torch.bfloat16, (m, n), "out"), m, k, sp, sb, _stream_ptr(stream),
         )
     )
     return out

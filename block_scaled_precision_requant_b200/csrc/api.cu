@@ -124,7 +124,9 @@ int64_t a_scale_ld(int64_t m) { return (m + 3) / 4 * 4; }
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
-                     uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream) {
+                     uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream,
+                     int64_t ldo = -1) {
+  if (ldo < 0) ldo = n;
   bsr_status st = check_dims(m, n, k, true, true);
   if (st != BSR_OK) return st;
   if (k % 128 != 0) return fail(BSR_ESHAPE, "bsr_gemm needs K %% 128 == 0 (K=%lld)", (long long)k);
@@ -148,20 +150,59 @@ bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w
       (st = encode_2d(&maps.as, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a_scale_t, m, nb, a_scale_ld(m) * 4, 128, 4,
                       CU_TENSOR_MAP_SWIZZLE_NONE, "a_scale_t")) != BSR_OK)
     return st;
-  return cuda_status(bsr::launch_gemm(maps, out, partials, d.status, (int)m, (int)n, (int)k, as_stream(stream), d.num_sms),
+  return cuda_status(bsr::launch_gemm(maps, out, partials, d.status, (int)m, (int)n, (int)k, (long long)ldo,
+                                      as_stream(stream), d.num_sms),
                      "gemm launch");
 }
 
-bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
-                       int64_t n, int64_t k, void* stream, int static_weight = 0) {
+bsr_status decode_segs_impl(const uint16_t* a, const bsr::DecodeSegs& segs, uint16_t* out, int64_t m, int64_t k,
+                            void* stream, int static_weight) {
   DevInfo d;
   bsr_status st;
   if ((st = device_info(d)) != BSR_OK) return st;
   const int mr = bsr::decode_rows_per_cta((int)m, (int)k, d.smem_optin);
   if (mr == 0) return fail(BSR_ESHAPE, "K=%lld too large for the decode kernel's shared memory", (long long)k);
-  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, static_weight, d.status,
-                                        d.smem_optin, as_stream(stream), d.num_sms),
+  return cuda_status(bsr::launch_decode(a, segs, out, (int)m, (int)k, mr, static_weight, d.status, d.smem_optin,
+                                        as_stream(stream), d.num_sms),
                      "decode launch");
+}
+
+bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
+                       int64_t n, int64_t k, void* stream, int static_weight = 0) {
+  bsr::DecodeSegs segs = {};
+  segs.count = 1;
+  segs.off[0] = 0;
+  segs.off[1] = (int)n;
+  segs.w[0] = w_i8;
+  segs.ws[0] = w_scale;
+  return decode_segs_impl(a, segs, out, m, k, stream, static_weight);
+}
+
+static_assert(BSR_MAX_SEGMENTS == bsr::kMaxDecodeSegs, "segment table size");
+
+// Validates a stacked weight (host arrays of num_segs device pointers and
+// row counts) and fills the decode segment table; total rows into n_total.
+bsr_status stacked_segs(const int8_t* const* w_i8, const float* const* w_scale, const int64_t* n_segs,
+                        int num_segs, bsr::DecodeSegs& segs, int64_t& n_total) {
+  if (num_segs < 1 || num_segs > BSR_MAX_SEGMENTS)
+    return fail(BSR_EINVAL, "num_segs %d not in [1, %d]", num_segs, BSR_MAX_SEGMENTS);
+  if (!w_i8 || !w_scale || !n_segs) return fail(BSR_EINVAL, "null segment array");
+  segs = {};
+  segs.count = num_segs;
+  n_total = 0;
+  for (int s = 0; s < num_segs; ++s) {
+    if (n_segs[s] < 0) return fail(BSR_EINVAL, "segment %d: negative row count", s);
+    if (n_segs[s] > 0 && (!w_i8[s] || !w_scale[s])) return fail(BSR_EINVAL, "segment %d: null pointer", s);
+    if (!aligned16(w_i8[s]) || !aligned16(w_scale[s]))
+      return fail(BSR_EALIGN, "segment %d: pointers must be 16-byte aligned", s);
+    segs.off[s] = (int)n_total;
+    segs.w[s] = w_i8[s];
+    segs.ws[s] = w_scale[s];
+    n_total += n_segs[s];
+    if (n_total > 2147483647LL) return fail(BSR_EINVAL, "stacked rows exceed 2^31 - 1");
+  }
+  segs.off[num_segs] = (int)n_total;
+  return BSR_OK;
 }
 
 bsr_status check_proj_args(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out) {
@@ -347,6 +388,54 @@ bsr_status bsr_proj_silu(const uint16_t* gate, const uint16_t* up, const int8_t*
   float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
   if ((st = bsr_requant_silu_a(gate, up, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
   return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
+}
+
+bsr_status bsr_decode_stacked(const uint16_t* a, const int8_t* const* w_i8, const float* const* w_scale,
+                              const int64_t* n_segs, int num_segs, uint16_t* out, int64_t m, int64_t k, unsigned flags,
+                              void* stream) {
+  if (flags & ~(unsigned)BSR_DECODE_STATIC_WEIGHT)
+    return fail(BSR_EINVAL, "bsr_decode_stacked: unknown flags 0x%x", flags);
+  bsr::DecodeSegs segs;
+  int64_t n = 0;
+  bsr_status st = stacked_segs(w_i8, w_scale, n_segs, num_segs, segs, n);
+  if (st != BSR_OK) return st;
+  if ((st = check_dims(m, n, k, true, true)) != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if (!a || !out) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(a) || (reinterpret_cast<uintptr_t>(out) & 1u))
+    return fail(BSR_EALIGN, "a must be 16-byte aligned, out 2-byte aligned");
+  return decode_segs_impl(a, segs, out, m, k, stream, (flags & BSR_DECODE_STATIC_WEIGHT) ? 1 : 0);
+}
+
+bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const float* const* w_scale,
+                            const int64_t* n_segs, int num_segs, uint16_t* out, int64_t m, int64_t k, void* scratch,
+                            size_t scratch_bytes, void* stream) {
+  bsr::DecodeSegs segs;
+  int64_t n = 0;
+  bsr_status st = stacked_segs(w_i8, w_scale, n_segs, num_segs, segs, n);
+  if (st != BSR_OK) return st;
+  if ((st = check_dims(m, n, k, true, true)) != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if (!a || !out) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(a) || (reinterpret_cast<uintptr_t>(out) & 1u))
+    return fail(BSR_EALIGN, "a must be 16-byte aligned, out 2-byte aligned");
+  if (m <= BSR_DECODE_MAX_M || k % 128 != 0) return decode_segs_impl(a, segs, out, m, k, stream, 0);
+  const size_t need = bsr_proj_scratch_bytes(m, k);
+  if (!scratch || scratch_bytes < need)
+    return fail(BSR_ESCRATCH, "scratch of %zu bytes needed, %zu given", need, scratch ? scratch_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
+  int8_t* a_i8 = static_cast<int8_t*>(scratch);
+  float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
+  if ((st = bsr_requant_a(a, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
+  // one GEMM per segment into its column slice of out (row stride = all rows)
+  for (int s = 0; s < num_segs; ++s) {
+    const int64_t ns = segs.off[s + 1] - segs.off[s];
+    if (ns == 0) continue;
+    if ((st = gemm_impl(a_i8, a_scale_t, w_i8[s], w_scale[s], out + segs.off[s], nullptr, m, ns, k, stream, n)) !=
+        BSR_OK)
+      return st;
+  }
+  return BSR_OK;
 }
 
 }  // extern "C"

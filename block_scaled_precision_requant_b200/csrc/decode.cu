@@ -80,11 +80,20 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int mr, int k, int nwar
 // MR: activation rows per CTA (compile time, >= rows actually present).
 template <int MR>
 __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
-    decode_kernel(const uint16_t* __restrict__ a, const int8_t* __restrict__ w_i8, const float* __restrict__ w_scale,
-                  __nv_bfloat16* __restrict__ out, int m, int n, int k, int scale_bulk, int static_weight,
-                  int* __restrict__ status) {
+    decode_kernel(const uint16_t* __restrict__ a, const DecodeSegs segs, __nv_bfloat16* __restrict__ out, int m,
+                  int k, int scale_bulk, int static_weight, int* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int nb = k >> 5;
+  const int n = segs.off[segs.count];  // output columns = rows of all segments
+  // codes and scales of output column r: row r - off[s] of its segment s
+  auto seg_row = [&](int r, const int8_t*& wr, const float*& wsr) {
+    int s = 0;
+#pragma unroll
+    for (int i = 1; i < kMaxDecodeSegs; ++i) s += (i < segs.count && r >= segs.off[i]) ? 1 : 0;
+    const size_t local = (size_t)(r - segs.off[s]);
+    wr = segs.w[s] + local * (size_t)k;
+    wsr = segs.ws[s] + local * (size_t)nb;
+  };
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
@@ -112,12 +121,15 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
   // of the weight is still streaming.
   auto issue_row = [&](int r) {
     if (lane == 0 && r < n) {
+      const int8_t* wr;
+      const float* wsr;
+      seg_row(r, wr, wsr);
       for (uint32_t c = 0; c < L.chunks; ++c) {
         const uint32_t blocks = min(32u, (uint32_t)nb - 32u * c);
         const uint32_t wb = blocks * 32u, sb = L.wscale_bytes ? blocks * 4u : 0u;
         mbar_arrive_expect_tx(&bars[c], wb + sb);
-        bulk_load(s_w + (size_t)c * 1024, w_i8 + (size_t)r * k + (size_t)c * 1024, wb, &bars[c]);
-        if (sb) bulk_load(s_ws + (size_t)c * 32, w_scale + (size_t)r * nb + (size_t)c * 32, sb, &bars[c]);
+        bulk_load(s_w + (size_t)c * 1024, wr + (size_t)c * 1024, wb, &bars[c]);
+        if (sb) bulk_load(s_ws + (size_t)c * 32, wsr + (size_t)c * 32, sb, &bars[c]);
       }
     }
   };
@@ -182,6 +194,10 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
   uint32_t phase = 0;
   bool aborted = false;
   for (; row < n; row += row_step) {
+    const int8_t* wrow;
+    const float* wsrow;
+    seg_row(row, wrow, wsrow);
+    (void)wrow;
     float acc[MR];
 #pragma unroll
     for (int r = 0; r < MR; ++r) acc[r] = 0.0f;
@@ -194,7 +210,7 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
       const uint4* wsrc = reinterpret_cast<const uint4*>(s_w + (size_t)b * 32);
       const uint4 w0 = wsrc[h];
       const uint4 w1 = wsrc[1 - h];
-      const float wsb = L.wscale_bytes ? s_ws[b] : __ldg(w_scale + (size_t)row * nb + b);
+      const float wsb = L.wscale_bytes ? s_ws[b] : __ldg(wsrow + b);
 #pragma unroll
       for (int r = 0; r < MR; ++r) {
         const uint4* cs = reinterpret_cast<const uint4*>(s_codes + (size_t)r * k + (size_t)b * 32);
@@ -246,9 +262,10 @@ int decode_rows_per_cta(int m, int k, size_t smem_limit) {
 }
 
 template <int MR>
-static cudaError_t launch_decode_t(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m,
-                                   int n, int k, int static_weight, int* status, size_t smem_limit,
-                                   cudaStream_t stream, int num_sms) {
+static cudaError_t launch_decode_t(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k,
+                                   int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                                   int num_sms) {
+  const int n = segs.off[segs.count];
   auto kern = decode_kernel<MR>;
   const bool sb = decode_scale_bulk(k);
   // Warps (= weight rows in flight) per CTA: spread the rows over all SMs,
@@ -285,21 +302,20 @@ static cudaError_t launch_decode_t(const uint16_t* a, const int8_t* w_i8, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
-  e = cudaLaunchKernelEx(&cfg, kern, a, w_i8, w_scale, o, m, n, k, sb ? 1 : 0, static_weight ? 1 : 0, status);
+  e = cudaLaunchKernelEx(&cfg, kern, a, segs, o, m, k, sb ? 1 : 0, static_weight ? 1 : 0, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
-                          int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
-                          int num_sms) {
+cudaError_t launch_decode(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k, int mr,
+                          int static_weight, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
   const int sw = static_weight;
   switch (mr) {
-    case 1: return launch_decode_t<1>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
-    case 2: return launch_decode_t<2>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
-    case 4: return launch_decode_t<4>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
-    case 8: return launch_decode_t<8>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
-    case 16: return launch_decode_t<16>(a, w_i8, w_scale, out, m, n, k, sw, status, smem_limit, stream, num_sms);
+    case 1: return launch_decode_t<1>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 2: return launch_decode_t<2>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 4: return launch_decode_t<4>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 8: return launch_decode_t<8>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 16: return launch_decode_t<16>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                 const __grid_constant__ CUtensorMap tm_ws, const __grid_constant__ CUtensorMap tm_as,
                 __nv_bfloat16* __restrict__ out, int32_t* __restrict__ partials, int* __restrict__ status, int m,
-                int n, int k, int n_tiles, int m_tiles, int m_fastest) {
+                int n, int k, int n_tiles, int m_tiles, int m_fastest, long long ldo) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled tiles, keeping the pointer
   // derived from the shared array so accesses stay shared-space loads
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               for (int k = 0; k < 8; ++k) {
                 const int mm = mr + 4 * k;
                 const float v = (i & 1) ? acc[i >> 1][k].y : acc[i >> 1][k].x;
-                if (mm < m) out[(size_t)mm * n + nn] = __float2bfloat16_rn(v);
+                if (mm < m) out[(size_t)mm * (size_t)ldo + nn] = __float2bfloat16_rn(v);
               }
             }
           }
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 size_t gemm_smem_bytes() { return gemm::SMEM_BYTES; }
 
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
-                        cudaStream_t stream, int num_sms) {
+                        long long ldo, cudaStream_t stream, int num_sms) {
   using namespace gemm;
   const int n_tiles = (n + BN - 1) / BN;
   const int m_tiles = (m + BM - 1) / BM;
@@ -466,7 +466,7 @@ cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, 
     }
     gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(maps.w, maps.a, maps.ws, maps.as,
                                                              reinterpret_cast<__nv_bfloat16*>(out), partials,
-                                                             status, m, n, k, n_tiles, m_tiles, m_fastest);
+                                                             status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
   } else {
     if (!granted[dev][0]) {
       e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
@@ -475,7 +475,7 @@ cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, 
     }
     gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(maps.w, maps.a, maps.ws, maps.as,
                                                               reinterpret_cast<__nv_bfloat16*>(out), nullptr,
-                                                              status, m, n, k, n_tiles, m_tiles, m_fastest);
+                                                              status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
   }
   return cudaGetLastError();
 }

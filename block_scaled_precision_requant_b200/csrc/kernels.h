@@ -19,13 +19,25 @@ cudaError_t launch_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, flo
                              float* w_scale, long long n, long long k, cudaStream_t stream, int num_sms);
 cudaError_t launch_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, int m, int k, int ld,
                              cudaStream_t stream, int num_sms);
+// Weight segments of one decode launch: output column r (global row of the
+// stacked weight) belongs to the segment s with off[s] <= r < off[s + 1] and
+// reads row r - off[s] of that segment's own codes and scales.
+constexpr int kMaxDecodeSegs = 8;
+struct DecodeSegs {
+  int count;
+  int off[kMaxDecodeSegs + 1];
+  const int8_t* w[kMaxDecodeSegs];
+  const float* ws[kMaxDecodeSegs];
+};
+
 int decode_rows_per_cta(int m, int k, size_t smem_limit);
-cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
-                          int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
-                          int num_sms);
+cudaError_t launch_decode(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k, int mr,
+                          int static_weight, int* status, size_t smem_limit, cudaStream_t stream, int num_sms);
 size_t gemm_smem_bytes();
+// out row stride ldo (elements) >= n: the output may be a column slice of a
+// wider matrix.
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
-                        cudaStream_t stream, int num_sms);
+                        long long ldo, cudaStream_t stream, int num_sms);
 
 // SiLU.mul: x = bf16(silu(g) * u) (x, g, u [M, K] BF16), and the fused
 // quantiser requant_a(bf16(silu(g) * u)) into the requant_a layout.

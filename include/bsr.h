@@ -184,6 +184,31 @@ bsr_status bsr_decode_ex(const uint16_t* a, const int8_t* w_i8, const float* w_s
                          int64_t n, int64_t k, unsigned flags, void* stream);
 
 /*
+ * Stacked weights (w8a8_decode/parts.rs, `W8a8Weight`: a weight stacked from
+ * segments, e.g. Q, K and V, whose `segment(i)` "writes the bits the stacked
+ * launch writes for those rows").  Segment s is a weight of its own
+ * (w_i8[s] [n_segs[s], K], w_scale[s] [n_segs[s], K/32], each 16-byte
+ * aligned, anywhere in device memory); the host arrays w_i8, w_scale and
+ * n_segs hold num_segs (1..BSR_MAX_SEGMENTS) entries.  The output is
+ * out [M, N] BF16 with N = sum of n_segs: segment s fills columns
+ * [off_s, off_s + n_segs[s]), off_s the sum of the earlier counts, with the
+ * bits a launch on that segment alone writes.
+ */
+#define BSR_MAX_SEGMENTS 8
+
+/* The decode kernel over all segments in one launch (flags as bsr_decode_ex). */
+bsr_status bsr_decode_stacked(const uint16_t* a, const int8_t* const* w_i8, const float* const* w_scale,
+                              const int64_t* n_segs, int num_segs, uint16_t* out, int64_t m, int64_t k, unsigned flags,
+                              void* stream);
+
+/* bsr_proj over a stacked weight: M <= BSR_DECODE_MAX_M (or K % 128 != 0):
+ * one decode launch over all segments; otherwise requant_a once into scratch
+ * (bsr_proj_scratch_bytes(M, K)) and one tensor-core GEMM per segment. */
+bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const float* const* w_scale,
+                            const int64_t* n_segs, int num_segs, uint16_t* out, int64_t m, int64_t k, void* scratch,
+                            size_t scratch_bytes, void* stream);
+
+/*
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
  * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:
  *   x = bf16_rne(silu(g) * u),  silu(g) = g / (1 + exp(-g)),

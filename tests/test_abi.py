@@ -83,6 +83,20 @@ def test_decode_ex_rejects_unknown_flags(L):
     assert "flags" in bsr.last_error()
 
 
+def test_stacked_argument_errors(L):
+    arr = (ctypes.c_void_p * 1)(_fake(256).value)
+    n1 = (ctypes.c_int64 * 1)(8)
+    assert L.bsr_decode_stacked(_fake(256), arr, arr, n1, 0, _fake(256), 1, 64, 0, None) == 1
+    assert "num_segs" in bsr.last_error()
+    assert L.bsr_decode_stacked(_fake(256), arr, arr, n1, 9, _fake(256), 1, 64, 0, None) == 1
+    assert L.bsr_proj_stacked(_fake(256), None, arr, n1, 1, _fake(256), 1, 64, None, 0, None) == 1
+    bad = (ctypes.c_void_p * 1)(_fake(264).value)
+    assert L.bsr_decode_stacked(_fake(256), bad, arr, n1, 1, _fake(256), 1, 64, 0, None) == 2
+    neg = (ctypes.c_int64 * 1)(-1)
+    assert L.bsr_decode_stacked(_fake(256), arr, arr, neg, 1, _fake(256), 1, 64, 0, None) == 1
+    assert L.bsr_decode_stacked(_fake(256), arr, arr, n1, 1, _fake(256), 1, 64, 4, None) == 1
+
+
 def test_scratch_errors(L):
     m, k = 64, 256
     need = L.bsr_proj_scratch_bytes(m, k)
