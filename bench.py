@@ -514,6 +514,65 @@ def prefill_extra(name, device, steps, warmup, peaks):
     return res
 
 
+def stacked_decode_extra(device, steps, peaks):
+    """Decode over a stacked weight shaped like Q, K and V of a grouped-query
+    layer (4096 + 1024 + 1024 rows, K = 4096, M = 1): one stacked launch per
+    step against one launch per segment, each a CUDA-graph loop over
+    rotating weight copies (>= 3x L2), static-weight option on."""
+    import torch
+
+    import block_scaled_precision_requant_b200 as bsr
+    from block_scaled_precision_requant_b200 import synth
+
+    k, ns = 4096, (4096, 1024, 1024)
+    a = torch.from_numpy(synth.make_activations(1, k, 1, "normal_outlier_channels")[0].view(np.int16)).view(
+        torch.bfloat16).to(device)
+    segs = []
+    for i, n in enumerate(ns):
+        w = synth.make_weight(n, k, 1 + i)
+        segs.append(bsr.requant_w(torch.from_numpy(w["w_packed"]).to(device), torch.from_numpy(w["w_e4m3"]).to(device),
+                                  float(w["scale2"])))
+    nbytes = sum(n * k + n * k // 8 + 2 * n for n in ns) + 2 * k
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(2, -(-3 * l2 // nbytes))
+    sets = [[(w.clone(), s.clone()) for w, s in segs] for _ in range(copies)]
+    out = torch.empty((1, sum(ns)), dtype=torch.bfloat16, device=device)
+    offs = np.cumsum((0,) + ns)
+
+    def stacked(i):
+        bsr.decode_stacked(a, sets[i % copies], out, static_weight=True)
+
+    def separate(i):
+        for j, (w, s) in enumerate(sets[i % copies]):
+            bsr.decode(a, w, s, out[:, offs[j]:offs[j + 1]], static_weight=True)
+
+    res = {}
+    for name, fn in (("stacked", stacked), ("separate", separate)):
+        for i in range(3):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(steps):
+                fn(i)
+        g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / steps
+        res[name] = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 /
+                     peaks["hbm_gbs"]}
+        del g
+    res["segments"] = list(ns)
+    res["bytes_per_step"] = nbytes
+    del sets
+    torch.cuda.empty_cache()
+    return res
+
+
 def silu_extra(g, steps, warmup):
     """The down projection from gate/up activations: the fused SiLU.mul
     quantiser + GEMM against the unfused SiLU.mul + requant_a + GEMM."""
@@ -621,6 +680,8 @@ def gpu_main(args):
             if name != args.workload:
                 extra[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks)
         line["prefill"] = extra
+        if decode:
+            line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks)
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
     if rank == 0:

@@ -65,6 +65,7 @@ __all__ = [
     "exp_f32",
     "silu_mul_bf16",
     "requant_silu_a",
+    "w4a16_gemv",
 ]
 
 GROUP = 32  # elements per int8 scale group
@@ -310,3 +311,22 @@ def silu_mul_bf16(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
 def requant_silu_a(g_bits: np.ndarray, u_bits: np.ndarray):
     """The SiLU.mul quantiser: requant_a of silu_mul_bf16(g, u)."""
     return requant_a(silu_mul_bf16(g_bits, u_bits))
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 W4A16 decode GEMV (gemv_sw.rs: `w4a16_gemv` / `w4a16_gemv_sw`, the
+# decode GEMV launched with the BF16 input, the packed E2M1 weight, its E4M3
+# scales, the F32 scale_2, the BF16 output, n and k).  The page gives the
+# arguments, not the arithmetic.  Reading taken: the weight is dequantised as
+# in requant_w (v = (e2m1 * e4m3) * scale2) and
+#     out[m, n] = bf16_rne( sum_k float(A[m, k]) * v[n, k] ),
+# with the sum taken here in float64 (the exact reference of any float32
+# summation order; a GPU result is compared within the BF16 tolerance).
+# ---------------------------------------------------------------------------
+
+
+def w4a16_gemv(a_bits, w_packed, w_e4m3, scale2, k: int) -> np.ndarray:
+    """BF16 output bits [M, N] of the W4A16 GEMV (float64 sum)."""
+    v = dequant_nvfp4(w_packed, w_e4m3, scale2, k).astype(np.float64)
+    x = bf16_bits_to_f32(np.atleast_2d(np.asarray(a_bits, dtype=np.uint16))).astype(np.float64)
+    return bf16_rne((x @ v.T).astype(np.float32))

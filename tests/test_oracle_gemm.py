@@ -164,3 +164,37 @@ def test_power_of_two_activation_scaling(tiny):
     out = oracle.bf16_bits_to_f32(oracle.proj_rows(tiny["a_bits"], w_i8, w_scale))
     out4 = oracle.bf16_bits_to_f32(oracle.proj_rows(x4.astype(np.uint16), w_i8, w_scale))
     assert np.array_equal(out4, out * np.float32(4.0))
+
+
+def test_w4a16_gemv_brute_force_tiny():
+    # brute force over the nibbles and scales, written out per element from the
+    # E2M1 / E4M3 tables, against the oracle's vectorised dequantise-and-sum
+    rng = np.random.default_rng(17)
+    n, k = 3, 64
+    w = synth.make_weight(n, k, seed=17)
+    a_bits = oracle.bf16_rne(rng.standard_normal((2, k)).astype(np.float32))
+    got = oracle.bf16_bits_to_f32(oracle.w4a16_gemv(a_bits, w["w_packed"], w["w_e4m3"], w["scale2"], k))
+    mags = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for r in range(2):
+        for j in range(n):
+            total = 0.0
+            for c in range(k):
+                byte = int(w["w_packed"][j, c // 2])
+                nib = (byte >> (4 * (c % 2))) & 0xF
+                e2 = mags[nib & 7] * (-1.0 if nib & 8 else 1.0)
+                s16 = float(oracle.e4m3_decode(np.array([w["w_e4m3"][j, c // 16]], dtype=np.uint8))[0])
+                v = np.float32(np.float32(e2 * s16) * np.float32(w["scale2"]))
+                total += float(oracle.bf16_bits_to_f32(np.array([a_bits[r, c]], dtype=np.uint16))[0]) * float(v)
+            want = oracle.bf16_bits_to_f32(oracle.bf16_rne(np.array([total], dtype=np.float32)))[0]
+            assert got[r, j] == want
+
+
+def test_w4a16_gemv_close_to_int8_projection():
+    # both read the same NVFP4 weight: the int8 projection differs from the
+    # exact W4A16 product only by the requantisation errors (a few percent)
+    w = synth.make_weight(64, 512, seed=18)
+    a_bits, _ = synth.make_activations(4, 512, 19, "normal")
+    x = oracle.bf16_bits_to_f32(oracle.w4a16_gemv(a_bits, w["w_packed"], w["w_e4m3"], w["scale2"], 512))
+    y = oracle.bf16_bits_to_f32(oracle.proj(a_bits, w["w_packed"], w["w_e4m3"], w["scale2"], 512))
+    rel = np.linalg.norm(x - y) / np.linalg.norm(x)
+    assert 0 < rel < 0.05
