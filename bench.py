@@ -573,6 +573,39 @@ def stacked_decode_extra(device, steps, peaks):
     return res
 
 
+def w4a16_extra(g, steps):
+    """The NVFP4 W4A16 decode GEMV on the decode workload's weight as stored
+    (0.5625 B per weight element): a CUDA-graph loop over rotating copies
+    (>= 3x L2), bytes = N*K*0.5625 + 2MK + 2MN per step."""
+    torch, bsr = g.torch, g.bsr
+    m, n, k = g.wl.shape
+    nbytes = n * k // 2 + n * k // 16 + 2 * m * k + 2 * m * n
+    l2 = torch.cuda.get_device_properties(g.dev).L2_cache_size
+    copies = max(2, -(-3 * l2 // nbytes))
+    ws = [(g.wp.clone(), g.we.clone()) for _ in range(copies)]
+    s2 = float(g.host["scale2"])
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=g.dev)
+    for i in range(3):
+        bsr.w4a16_decode(g.a, *ws[i % copies], s2, out)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for i in range(steps):
+            bsr.w4a16_decode(g.a, *ws[i % copies], s2, out)
+    gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del gr, ws
+    g.check_status()
+    return {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
+            "note": "reads the NVFP4 weight as stored; not bit-compatible with the int8 path"}
+
+
 def silu_extra(g, steps, warmup):
     """The down projection from gate/up activations: the fused SiLU.mul
     quantiser + GEMM against the unfused SiLU.mul + requant_a + GEMM."""
@@ -634,6 +667,7 @@ def gpu_main(args):
         kernel = "gemm_kernel"
     t_rw = g.timed_requant_w_only(min(args.steps, 20), args.warmup)
     g.check_status()
+    w4 = w4a16_extra(g, max(args.steps, 20)) if decode and not args.no_extra and world == 1 else None
 
     ms_step, ms_e2e, ms_kernel, ms_rw = dist_max(
         [mean_ms(t_steps), mean_ms(t_e2e), mean_ms(t_kernel), mean_ms(t_rw)], device="cuda" if world > 1 else "cpu")
@@ -680,6 +714,8 @@ def gpu_main(args):
             if name != args.workload:
                 extra[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks)
         line["prefill"] = extra
+        if w4 is not None:
+            line["w4a16_decode"] = w4
         if decode:
             line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks)
     if rank == 0 and world == 1 and not args.no_cpu:

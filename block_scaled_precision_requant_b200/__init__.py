@@ -49,6 +49,7 @@ __all__ = [
     "MAX_SEGMENTS",
     "decode_stacked",
     "proj_stacked",
+    "w4a16_decode",
     "silu_mul",
     "requant_silu_a",
     "proj_silu_scratch_bytes",
@@ -93,6 +94,7 @@ SIGNATURES = [
     ("bsr_decode_ex", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_decode_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_proj_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _P, ctypes.c_size_t, _P]),
+    ("bsr_w4a16_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
     ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
@@ -490,6 +492,29 @@ def proj_stacked(a, segments, out=None, scratch=None, stream=None):
             _dev(a, torch.bfloat16, (m, k), "a"), ctypes.cast(w_arr, ctypes.c_void_p),
             ctypes.cast(s_arr, ctypes.c_void_p), ctypes.cast(n_arr, ctypes.c_void_p), num,
             _dev(out, torch.bfloat16, (m, n), "out"), m, k, sp, sb, _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def w4a16_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
+    """NVFP4 W4A16 decode GEMV on the stored weight -> out [M, N] bfloat16."""
+    torch = _torch()
+    m, k = a.shape
+    n = w_packed.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    _check(
+        lib().bsr_w4a16_decode(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(w_packed, torch.uint8, (n, k // 2), "w_packed"),
+            _dev(w_e4m3, torch.uint8, (n, k // 16), "w_e4m3"),
+            ctypes.c_float(float(scale2)),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            _stream_ptr(stream),
         )
     )
     return out

@@ -438,4 +438,21 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
   return BSR_OK;
 }
 
+bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                            uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if (!a || !w_packed || !w_e4m3 || !out) return fail(BSR_EINVAL, "null pointer");
+  if (!aligned16(a) || !aligned16(w_packed) || !aligned16(w_e4m3) || (reinterpret_cast<uintptr_t>(out) & 1u))
+    return fail(BSR_EALIGN, "a, w_packed, w_e4m3 must be 16-byte aligned, out 2-byte aligned");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  if ((size_t)k * 2 > d.smem_optin)
+    return fail(BSR_ESHAPE, "K=%lld too large for one BF16 activation row in shared memory", (long long)k);
+  return cuda_status(bsr::launch_w4a16_decode(a, w_packed, w_e4m3, scale2, out, (int)m, (int)n, (int)k, d.smem_optin,
+                                              as_stream(stream), d.num_sms),
+                     "w4a16 decode launch");
+}
+
 }  // extern "C"

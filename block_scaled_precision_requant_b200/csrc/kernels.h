@@ -46,6 +46,11 @@ cudaError_t launch_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* x, i
 cudaError_t launch_requant_silu_a(const uint16_t* g, const uint16_t* u, int8_t* a_i8, float* a_scale_t, int m, int k,
                                   int ld, cudaStream_t stream, int num_sms);
 
+// NVFP4 W4A16 decode GEMV: out [M, N] = A [M, K] . dequant(W)^T, F32 sums.
+cudaError_t launch_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                                uint16_t* out, int m, int n, int k, size_t smem_limit, cudaStream_t stream,
+                                int num_sms);
+
 // Test entry: one CTA waits on an mbarrier nothing arrives on, through the
 // bounded wait of the pipelined kernels, for at most limit_ns.
 cudaError_t launch_debug_wait(int* status, unsigned long long limit_ns, cudaStream_t stream);

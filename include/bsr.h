@@ -209,6 +209,22 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
                             size_t scratch_bytes, void* stream);
 
 /*
+ * bsr_w4a16_decode -- gemv_sw.rs, `w4a16_gemv` / `w4a16_gemv_sw`: the
+ * NVFP4 W4A16 decode GEMV on the weight as stored (no requantisation).
+ *   a         [M, K]    BF16
+ *   w_packed  [N, K/2]  uint8, E2M1 pairs, element 2i in the low nibble of byte i
+ *   w_e4m3    [N, K/16] uint8, E4M3 scale of each 16-element block
+ *   scale2    per-tensor F32 scale (host value)
+ *   out       [M, N]    BF16: sum_k a * (e2m1 * e4m3) * scale2, float32 sums
+ * (per 16-block, then times the E4M3 scale, scale2 once at the end).  Not
+ * bit-compatible with bsr_proj (that path requantises to int8).  K > 0,
+ * K % 32 == 0, 2K bytes within the device's shared memory per CTA; pointers
+ * 16-byte aligned (out 2-byte).  Any M; built for M <= 16.
+ */
+bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                            uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
+
+/*
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
  * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:
  *   x = bf16_rne(silu(g) * u),  silu(g) = g / (1 + exp(-g)),
