@@ -155,30 +155,35 @@ bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w
                      "gemm launch");
 }
 
+bsr_status decode_mr(int64_t m, int64_t k, DevInfo& d, int& mr) {
+  bsr_status st;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  mr = bsr::decode_rows_per_cta((int)m, (int)k, d.smem_optin);
+  if (mr == 0) return fail(BSR_ESHAPE, "K=%lld too large for the decode kernel's shared memory", (long long)k);
+  return BSR_OK;
+}
+
 bsr_status decode_segs_impl(const uint16_t* a, const bsr::DecodeSegs& segs, uint16_t* out, int64_t m, int64_t k,
                             void* stream, int static_weight) {
   DevInfo d;
-  bsr_status st;
-  if ((st = device_info(d)) != BSR_OK) return st;
-  const int mr = bsr::decode_rows_per_cta((int)m, (int)k, d.smem_optin);
-  if (mr == 0) return fail(BSR_ESHAPE, "K=%lld too large for the decode kernel's shared memory", (long long)k);
-  return cuda_status(bsr::launch_decode(a, segs, out, (int)m, (int)k, mr, static_weight, d.status, d.smem_optin,
-                                        as_stream(stream), d.num_sms),
+  int mr = 0;
+  bsr_status st = decode_mr(m, k, d, mr);
+  if (st != BSR_OK) return st;
+  return cuda_status(bsr::launch_decode_stacked(a, segs, out, (int)m, (int)k, mr, static_weight, d.status,
+                                                d.smem_optin, as_stream(stream), d.num_sms),
                      "decode launch");
 }
 
 bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m,
                        int64_t n, int64_t k, void* stream, int static_weight = 0) {
-  bsr::DecodeSegs segs = {};
-  segs.count = 1;
-  segs.off[0] = 0;
-  segs.off[1] = (int)n;
-  segs.w[0] = w_i8;
-  segs.ws[0] = w_scale;
-  return decode_segs_impl(a, segs, out, m, k, stream, static_weight);
+  DevInfo d;
+  int mr = 0;
+  bsr_status st = decode_mr(m, k, d, mr);
+  if (st != BSR_OK) return st;
+  return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, static_weight, d.status,
+                                        d.smem_optin, as_stream(stream), d.num_sms),
+                     "decode launch");
 }
-
-static_assert(BSR_MAX_SEGMENTS == bsr::kMaxDecodeSegs, "segment table size");
 
 // Validates a stacked weight (host arrays of num_segs device pointers and
 // row counts) and fills the decode segment table; total rows into n_total.

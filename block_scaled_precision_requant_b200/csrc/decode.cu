@@ -77,23 +77,43 @@ __host__ __device__ inline DecodeSmem decode_smem_layout(int mr, int k, int nwar
   return L;
 }
 
+// Where a weight row comes from: one weight (compact kernel parameters: they
+// are read on the kernel's critical path before its first copy, and a larger
+// parameter block measured ~0.5 us slower per launch), or a table of up to
+// kMaxDecodeSegs segments (stacked weight).
+struct DecodeSingle {
+  const int8_t* w;
+  const float* ws;
+  int n;
+};
+__device__ __forceinline__ int src_rows(const DecodeSingle& s) { return s.n; }
+__device__ __forceinline__ int src_rows(const DecodeSegs& s) { return s.off[s.count]; }
+__device__ __forceinline__ void src_row(const DecodeSingle& s, int r, int k, int nb, const int8_t*& w,
+                                        const float*& ws) {
+  w = s.w + (size_t)r * (size_t)k;
+  ws = s.ws + (size_t)r * (size_t)nb;
+}
+// output column r of a stacked weight: row r - off[s] of the segment s with
+// off[s] <= r < off[s + 1]
+__device__ __forceinline__ void src_row(const DecodeSegs& s, int r, int k, int nb, const int8_t*& w,
+                                        const float*& ws) {
+  int i = 0;
+#pragma unroll
+  for (int j = 1; j < kMaxDecodeSegs; ++j) i += (j < s.count && r >= s.off[j]) ? 1 : 0;
+  const size_t local = (size_t)(r - s.off[i]);
+  w = s.w[i] + local * (size_t)k;
+  ws = s.ws[i] + local * (size_t)nb;
+}
+
 // MR: activation rows per CTA (compile time, >= rows actually present).
-template <int MR>
+template <int MR, class Src>
 __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
-    decode_kernel(const uint16_t* __restrict__ a, const DecodeSegs segs, __nv_bfloat16* __restrict__ out, int m,
-                  int k, int scale_bulk, int static_weight, int* __restrict__ status) {
+    decode_kernel(const uint16_t* __restrict__ a, const Src src, __nv_bfloat16* __restrict__ out, int m, int k,
+                  int scale_bulk, int static_weight, int* __restrict__ status) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int nb = k >> 5;
-  const int n = segs.off[segs.count];  // output columns = rows of all segments
-  // codes and scales of output column r: row r - off[s] of its segment s
-  auto seg_row = [&](int r, const int8_t*& wr, const float*& wsr) {
-    int s = 0;
-#pragma unroll
-    for (int i = 1; i < kMaxDecodeSegs; ++i) s += (i < segs.count && r >= segs.off[i]) ? 1 : 0;
-    const size_t local = (size_t)(r - segs.off[s]);
-    wr = segs.w[s] + local * (size_t)k;
-    wsr = segs.ws[s] + local * (size_t)nb;
-  };
+  const int n = src_rows(src);  // output columns = weight rows
+  auto seg_row = [&](int r, const int8_t*& wr, const float*& wsr) { src_row(src, r, k, nb, wr, wsr); };
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
@@ -261,12 +281,11 @@ int decode_rows_per_cta(int m, int k, size_t smem_limit) {
   return fits(mr) ? mr : 0;
 }
 
-template <int MR>
-static cudaError_t launch_decode_t(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k,
+template <int MR, class Src>
+static cudaError_t launch_decode_t(const uint16_t* a, const Src& src, int n, uint16_t* out, int m, int k,
                                    int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
                                    int num_sms) {
-  const int n = segs.off[segs.count];
-  auto kern = decode_kernel<MR>;
+  auto kern = decode_kernel<MR, Src>;
   const bool sb = decode_scale_bulk(k);
   // Warps (= weight rows in flight) per CTA: spread the rows over all SMs,
   // at most decode_max_warps<MR>() per CTA and as many row slots as fit in
@@ -276,7 +295,7 @@ static cudaError_t launch_decode_t(const uint16_t* a, const DecodeSegs& segs, ui
   w = w < 1 ? 1 : (w > kMaxW ? kMaxW : w);
   while (w > 1 && decode_smem_layout(MR, k, w, sb).total > smem_limit) --w;
   const size_t smem = decode_smem_layout(MR, k, w, sb).total;
-  // dynamic shared-memory limit granted so far, per device
+  // dynamic shared-memory limit granted so far, per device (per <MR, Src>)
   static size_t granted[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -302,22 +321,36 @@ static cudaError_t launch_decode_t(const uint16_t* a, const DecodeSegs& segs, ui
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
-  e = cudaLaunchKernelEx(&cfg, kern, a, segs, o, m, k, sb ? 1 : 0, static_weight ? 1 : 0, status);
+  e = cudaLaunchKernelEx(&cfg, kern, a, src, o, m, k, sb ? 1 : 0, static_weight ? 1 : 0, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k, int mr,
-                          int static_weight, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
-  const int sw = static_weight;
+template <class Src>
+static cudaError_t launch_decode_src(const uint16_t* a, const Src& src, int n, uint16_t* out, int m, int k, int mr,
+                                     int sw, int* status, size_t smem_limit, cudaStream_t stream, int num_sms) {
   switch (mr) {
-    case 1: return launch_decode_t<1>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
-    case 2: return launch_decode_t<2>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
-    case 4: return launch_decode_t<4>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
-    case 8: return launch_decode_t<8>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
-    case 16: return launch_decode_t<16>(a, segs, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 1: return launch_decode_t<1, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 2: return launch_decode_t<2, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 4: return launch_decode_t<4, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 8: return launch_decode_t<8, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
+    case 16: return launch_decode_t<16, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
+                          int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                          int num_sms) {
+  const DecodeSingle src = {w_i8, w_scale, n};
+  return launch_decode_src(a, src, n, out, m, k, mr, static_weight, status, smem_limit, stream, num_sms);
+}
+
+cudaError_t launch_decode_stacked(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k, int mr,
+                                  int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                                  int num_sms) {
+  return launch_decode_src(a, segs, segs.off[segs.count], out, m, k, mr, static_weight, status, smem_limit, stream,
+                           num_sms);
 }
 
 }  // namespace bsr

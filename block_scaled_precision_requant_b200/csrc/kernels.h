@@ -31,8 +31,12 @@ struct DecodeSegs {
 };
 
 int decode_rows_per_cta(int m, int k, size_t smem_limit);
-cudaError_t launch_decode(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k, int mr,
-                          int static_weight, int* status, size_t smem_limit, cudaStream_t stream, int num_sms);
+cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
+                          int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                          int num_sms);
+cudaError_t launch_decode_stacked(const uint16_t* a, const DecodeSegs& segs, uint16_t* out, int m, int k, int mr,
+                                  int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
+                                  int num_sms);
 size_t gemm_smem_bytes();
 // out row stride ldo (elements) >= n: the output may be a column slice of a
 // wider matrix.
