@@ -523,7 +523,7 @@ def mean_ms(times):
     return float(np.mean(times))
 
 
-def prefill_extra(name, device, steps, warmup, peaks):
+def prefill_extra(name, device, steps, warmup, peaks, cpu=True):
     """Secondary measurement of one prefill workload (rank-local)."""
     g = Gpu(name, device)
     m, n, k = g.wl.shape
@@ -546,7 +546,7 @@ def prefill_extra(name, device, steps, warmup, peaks):
         "ms": {"step": t_step, "gemm": t_gemm, "requant_a": t_ra, "requant_w": t_rw},
     }
     if g.wl.act == "silu_mul":
-        res["silu"] = silu_extra(g, steps, warmup)
+        res["silu"] = silu_extra(g, steps, warmup, cpu)
     del g
     import torch
 
@@ -554,7 +554,7 @@ def prefill_extra(name, device, steps, warmup, peaks):
     return res
 
 
-def stacked_decode_extra(device, steps, peaks):
+def stacked_decode_extra(device, steps, peaks, cpu=True):
     """Decode over a stacked weight shaped like Q, K and V of a grouped-query
     layer (4096 + 1024 + 1024 rows, K = 4096, M = 1): one stacked launch per
     step against one launch per segment, each a CUDA-graph loop over
@@ -608,12 +608,23 @@ def stacked_decode_extra(device, steps, peaks):
         del g
     res["segments"] = list(ns)
     res["bytes_per_step"] = nbytes
+    if cpu:
+        import oracle
+
+        a_bits = synth.make_activations(1, k, 1, "normal_outlier_channels")[0]
+        hw = []
+        for i, n in enumerate(ns):
+            w = synth.make_weight(n, k, 1 + i)
+            hw.append(oracle.requant_w(w["w_packed"], w["w_e4m3"], w["scale2"], k))
+        t, calls = oracle_seconds(lambda: [oracle.proj_rows(a_bits, wq, wsc) for wq, wsc in hw], 3.0)
+        res["cpu_baseline"] = {"kind": "oracle", "cores": 1, "gbs": nbytes / t / 1e9, "ms_per_step": t * 1e3,
+                               "sample": f"{calls} full step(s) over the three segments (M=1)"}
     del sets
     torch.cuda.empty_cache()
     return res
 
 
-def w4a16_extra(g, steps):
+def w4a16_extra(g, steps, cpu=True):
     """The NVFP4 W4A16 decode GEMV on the decode workload's weight as stored
     (0.5625 B per weight element): a CUDA-graph loop over rotating copies
     (>= 3x L2), bytes = N*K*0.5625 + 2MK + 2MN per step."""
@@ -642,11 +653,31 @@ def w4a16_extra(g, steps):
     ms = e0.elapsed_time(e1) / steps
     del gr, ws
     g.check_status()
-    return {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
-            "note": "reads the NVFP4 weight as stored; not bit-compatible with the int8 path"}
+    res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
+           "note": "reads the NVFP4 weight as stored; not bit-compatible with the int8 path"}
+    if cpu:
+        import oracle
+
+        hd = g.host
+        t, calls = oracle_seconds(lambda: oracle.w4a16_gemv(hd["a_bits"], hd["w_packed"], hd["w_e4m3"], hd["scale2"],
+                                                            k), 3.0)
+        res["cpu_baseline"] = {"kind": "oracle", "cores": 1, "gbs": nbytes / t / 1e9, "ms_per_step": t * 1e3,
+                               "sample": f"{calls} full step(s) (M={m})"}
+    return res
 
 
-def silu_extra(g, steps, warmup):
+def oracle_seconds(fn, budget_s, max_calls=50):
+    """Mean host seconds of fn() over calls bounded by budget_s."""
+    done, spent = 0, 0.0
+    while done < 1 or (spent < budget_s and done < max_calls):
+        t0 = time.perf_counter()
+        fn()
+        spent += time.perf_counter() - t0
+        done += 1
+    return spent / done, done
+
+
+def silu_extra(g, steps, warmup, cpu=True):
     """The down projection from gate/up activations: the fused SiLU.mul
     quantiser + GEMM against the unfused SiLU.mul + requant_a + GEMM."""
     torch, bsr = g.torch, g.bsr
@@ -656,6 +687,14 @@ def silu_extra(g, steps, warmup):
     gb, ub, _ = synth.make_gate_up(m, k, g.wl.seed)
     gate = torch.from_numpy(gb.view(np.int16)).view(torch.bfloat16).to(g.dev)
     up = torch.from_numpy(ub.view(np.int16)).view(torch.bfloat16).to(g.dev)
+    cpu_res = None
+    if cpu:
+        import oracle
+
+        rows = 4
+        t, calls = oracle_seconds(lambda: oracle.requant_silu_a(gb[:rows], ub[:rows]), 3.0)
+        cpu_res = {"kind": "oracle", "cores": 1, "requant_silu_a_gbs": rows * k * 5.125 / t / 1e9,
+                   "sample": f"requant_silu_a of {rows} rows x K={k}, {calls} call(s)"}
     del gb, ub
     x = torch.empty((m, k), dtype=torch.bfloat16, device=g.dev)
     scratch = torch.empty((bsr.proj_silu_scratch_bytes(m, k),), dtype=torch.uint8, device=g.dev)
@@ -672,6 +711,7 @@ def silu_extra(g, steps, warmup):
         "requant_silu_a_gbs": m * k * 5.125 / t_quant / 1e6,
         "silu_mul_gbs": m * k * 6 / t_mul / 1e6,
         "ms": {"proj_silu": t_fused, "silu_mul_then_proj": t_unfused, "requant_silu_a": t_quant, "silu_mul": t_mul},
+        "cpu_baseline": cpu_res,
     }
 
 
@@ -710,7 +750,8 @@ def gpu_main(args):
         kernel = "gemm_kernel"
     t_rw = g.timed_requant_w_only(min(args.steps, 20), args.warmup)
     g.check_status()
-    w4 = w4a16_extra(g, max(args.steps, 20)) if decode and not args.no_extra and world == 1 else None
+    w4 = (w4a16_extra(g, max(args.steps, 20), cpu=not args.no_cpu)
+          if decode and not args.no_extra and world == 1 else None)
 
     ms_step, ms_e2e, ms_kernel, ms_rw, ms_e2e_eager = dist_max(
         [mean_ms(t_steps), mean_ms(t_e2e), mean_ms(t_kernel), mean_ms(t_rw), mean_ms(t_e2e_eager)],
@@ -759,12 +800,13 @@ def gpu_main(args):
         extra = {}
         for name in ("ffn_up", "ffn_down", "square_ragged"):
             if name != args.workload:
-                extra[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks)
+                extra[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks,
+                                            cpu=not args.no_cpu)
         line["prefill"] = extra
         if w4 is not None:
             line["w4a16_decode"] = w4
         if decode:
-            line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks)
+            line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks, cpu=not args.no_cpu)
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
     if rank == 0:
