@@ -20,7 +20,11 @@ Sources (the launcher pages of the ``metrale_model_layers`` ops crate):
   bits do not depend on the row count or on the other rows.
 * ``w8a8_decode/parts.rs`` -- doc comment of ``W8a8Weight::segment``: a
   segment of a stacked weight yields the bits the stacked launch yields for
-  those rows.
+  those rows; ``W8a8Kernels::quant_silu``: the SiLU.mul quantiser (its
+  arithmetic is this module's reading, see ``silu_mul_bf16``).
+* ``gemv_sw.rs`` -- the ``w4a16_gemv`` / ``w4a16_gemv_sw`` launches: the NVFP4
+  W4A16 decode GEMV's arguments (its arithmetic is this module's reading, see
+  ``w4a16_gemv``).
 
 Conventions the pages leave open, fixed here (each is listed, with the reading
 taken, in the design notes of this repository):
