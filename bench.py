@@ -677,6 +677,57 @@ def oracle_seconds(fn, budget_s, max_calls=50):
     return spent / done, done
 
 
+def stacked_prefill_extra(device, steps, warmup):
+    """Prefill over a stacked weight shaped like Q, K and V of a grouped-query
+    layer (4096 + 1024 + 1024 rows, K = 4096, M = 2048): bsr_proj_stacked
+    (requant_a once, the segments' GEMMs concurrently with grids in
+    proportion to their tiles) against one bsr_proj per segment; L2 flushed
+    before every step."""
+    import torch
+
+    import block_scaled_precision_requant_b200 as bsr
+    from block_scaled_precision_requant_b200 import synth
+
+    m, k, ns = 2048, 4096, (4096, 1024, 1024)
+    a = torch.from_numpy(synth.make_activations(m, k, 2, "normal_outlier_channels")[0].view(np.int16)).view(
+        torch.bfloat16).to(device)
+    segs = []
+    for i, n in enumerate(ns):
+        w = synth.make_weight(n, k, 2 + i)
+        segs.append(bsr.requant_w(torch.from_numpy(w["w_packed"]).to(device), torch.from_numpy(w["w_e4m3"]).to(device),
+                                  float(w["scale2"])))
+    out = torch.empty((m, sum(ns)), dtype=torch.bfloat16, device=device)
+    outs = [torch.empty((m, n), dtype=torch.bfloat16, device=device) for n in ns]
+    scratch = torch.empty((bsr.proj_scratch_bytes(m, k),), dtype=torch.uint8, device=device)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.mean(ts))
+
+    t_st = timed(lambda: bsr.proj_stacked(a, segs, out, scratch))
+    t_sep = timed(lambda: [bsr.proj(a, w, s, o, scratch) for (w, s), o in zip(segs, outs)])
+    ops = 2 * m * sum(ns) * k
+    status = bsr.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    del segs, out, outs, scratch, flush
+    torch.cuda.empty_cache()
+    return {"segments": list(ns), "m": m, "k": k, "stacked": {"ms": t_st, "tops": ops / t_st / 1e9},
+            "separate": {"ms": t_sep, "tops": ops / t_sep / 1e9}}
+
+
 def silu_extra(g, steps, warmup, cpu=True):
     """The down projection from gate/up activations: the fused SiLU.mul
     quantiser + GEMM against the unfused SiLU.mul + requant_a + GEMM."""
@@ -805,6 +856,7 @@ def gpu_main(args):
         line["prefill"] = extra
         if w4 is not None:
             line["w4a16_decode"] = w4
+        line["stacked_prefill"] = stacked_prefill_extra(dev, min(args.steps, 10), 3)
         if decode:
             line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks, cpu=not args.no_cpu)
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -125,7 +125,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
                      uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream,
-                     int64_t ldo = -1) {
+                     int64_t ldo = -1, int max_ctas = 0) {
   if (ldo < 0) ldo = n;
   bsr_status st = check_dims(m, n, k, true, true);
   if (st != BSR_OK) return st;
@@ -151,7 +151,7 @@ bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w
                       CU_TENSOR_MAP_SWIZZLE_NONE, "a_scale_t")) != BSR_OK)
     return st;
   return cuda_status(bsr::launch_gemm(maps, out, partials, d.status, (int)m, (int)n, (int)k, (long long)ldo,
-                                      as_stream(stream), d.num_sms),
+                                      as_stream(stream), d.num_sms, max_ctas),
                      "gemm launch");
 }
 
@@ -183,6 +183,35 @@ bsr_status decode_impl(const uint16_t* a, const int8_t* w_i8, const float* w_sca
   return cuda_status(bsr::launch_decode(a, w_i8, w_scale, out, (int)m, (int)n, (int)k, mr, static_weight, d.status,
                                         d.smem_optin, as_stream(stream), d.num_sms),
                      "decode launch");
+}
+
+static_assert(BSR_MAX_SEGMENTS == bsr::kMaxDecodeSegs, "segment table size");
+
+// Side streams and events of the stacked tensor-core route, created once per
+// device; the enqueue sequence that uses them runs under a lock.
+struct StackedStreams {
+  bool ready = false;
+  cudaStream_t side[BSR_MAX_SEGMENTS] = {};
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join[BSR_MAX_SEGMENTS] = {};
+};
+StackedStreams g_stacked[64];
+std::mutex g_stacked_mu;
+
+bsr_status stacked_streams(int dev, StackedStreams*& out) {
+  if (dev < 0 || dev >= 64) return fail(BSR_ENODEV, "device index %d out of range", dev);
+  StackedStreams& ss = g_stacked[dev];
+  if (!ss.ready) {
+    cudaError_t e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+    for (int i = 0; e == cudaSuccess && i < BSR_MAX_SEGMENTS; ++i) {
+      e = cudaStreamCreateWithFlags(&ss.side[i], cudaStreamNonBlocking);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return fail(BSR_ECUDA, "stacked side streams: %s", cudaGetErrorString(e));
+    ss.ready = true;
+  }
+  out = &ss;
+  return BSR_OK;
 }
 
 // Validates a stacked weight (host arrays of num_segs device pointers and
@@ -432,13 +461,37 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
   int8_t* a_i8 = static_cast<int8_t*>(scratch);
   float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
   if ((st = bsr_requant_a(a, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
-  // one GEMM per segment into its column slice of out (row stride = all rows)
+  // One GEMM per segment into its column slice of out (row stride = all
+  // rows).  The segments run concurrently, each on a side stream forked from
+  // and joined back into the caller's stream, with persistent grids sized in
+  // proportion to their tile counts so that together they fill the SMs once
+  // (a small segment alone would leave most SMs idle).
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(BSR_ENODEV, "cudaGetDevice failed");
+  long long tiles[BSR_MAX_SEGMENTS] = {}, total_tiles = 0;
   for (int s = 0; s < num_segs; ++s) {
     const int64_t ns = segs.off[s + 1] - segs.off[s];
-    if (ns == 0) continue;
-    if ((st = gemm_impl(a_i8, a_scale_t, w_i8[s], w_scale[s], out + segs.off[s], nullptr, m, ns, k, stream, n)) !=
-        BSR_OK)
+    tiles[s] = ((ns + 127) / 128) * ((m + 127) / 128);
+    total_tiles += tiles[s];
+  }
+  std::lock_guard<std::mutex> lk(g_stacked_mu);
+  StackedStreams* ss = nullptr;
+  if ((st = stacked_streams(dev, ss)) != BSR_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  if (cudaEventRecord(ss->fork, cs) != cudaSuccess) return fail(BSR_ECUDA, "stacked fork record failed");
+  for (int s = 0; s < num_segs; ++s) {
+    if (tiles[s] == 0) continue;
+    int ctas = (int)((long long)d.num_sms * tiles[s] / total_tiles);
+    ctas = ctas < 1 ? 1 : ctas;
+    if (cudaStreamWaitEvent(ss->side[s], ss->fork, 0) != cudaSuccess) return fail(BSR_ECUDA, "stacked fork wait failed");
+    const int64_t ns = segs.off[s + 1] - segs.off[s];
+    if ((st = gemm_impl(a_i8, a_scale_t, w_i8[s], w_scale[s], out + segs.off[s], nullptr, m, ns, k, ss->side[s], n,
+                        ctas)) != BSR_OK)
       return st;
+    if (cudaEventRecord(ss->join[s], ss->side[s]) != cudaSuccess) return fail(BSR_ECUDA, "stacked join record failed");
+    if (cudaStreamWaitEvent(cs, ss->join[s], 0) != cudaSuccess) return fail(BSR_ECUDA, "stacked join wait failed");
   }
   return BSR_OK;
 }

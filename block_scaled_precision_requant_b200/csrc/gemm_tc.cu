@@ -443,12 +443,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 size_t gemm_smem_bytes() { return gemm::SMEM_BYTES; }
 
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
-                        long long ldo, cudaStream_t stream, int num_sms) {
+                        long long ldo, cudaStream_t stream, int num_sms, int max_ctas) {
   using namespace gemm;
   const int n_tiles = (n + BN - 1) / BN;
   const int m_tiles = (m + BM - 1) / BM;
   const int tiles = n_tiles * m_tiles;
-  const int grid = tiles < num_sms ? tiles : num_sms;
+  // persistent CTAs: one per SM, or fewer when the caller shares the GPU
+  // between concurrent launches (max_ctas)
+  const int cap = (max_ctas > 0 && max_ctas < num_sms) ? max_ctas : num_sms;
+  const int grid = tiles < cap ? tiles : cap;
   // Sweep the smaller operand fastest so that it stays resident in L2 while
   // the larger one streams through once.
   const int m_fastest = ((long long)m <= (long long)n) ? 1 : 0;

@@ -39,9 +39,10 @@ cudaError_t launch_decode_stacked(const uint16_t* a, const DecodeSegs& segs, uin
                                   int num_sms);
 size_t gemm_smem_bytes();
 // out row stride ldo (elements) >= n: the output may be a column slice of a
-// wider matrix.
+// wider matrix.  max_ctas > 0 caps the persistent grid (to share the GPU
+// between concurrent launches).
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
-                        long long ldo, cudaStream_t stream, int num_sms);
+                        long long ldo, cudaStream_t stream, int num_sms, int max_ctas = 0);
 
 // SiLU.mul: x = bf16(silu(g) * u) (x, g, u [M, K] BF16), and the fused
 // quantiser requant_a(bf16(silu(g) * u)) into the requant_a layout.
