@@ -32,6 +32,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -213,13 +214,18 @@ def roofline(bound, achieved, peak, unit, traffic):
 
 
 def kernel_source_hash():
-    """Hash of the CUDA sources: stored ncu traffic counts are valid only for it."""
+    """Hash of the CUDA sources with comments and whitespace removed: stored
+    ncu traffic counts are valid only for this code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_scaled_precision_requant_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # block comments
+        text = re.sub(r"//[^\n]*", " ", text)  # line comments (no source string holds //)
+        text = " ".join(text.split())
+        h.update(name.encode())
+        h.update(text.encode())
     return h.hexdigest()[:16]
 
 

@@ -8,13 +8,17 @@
 // l, l+32, ...) and the 32 lane sums are added in a fixed xor tree, so an
 // output's bits depend only on K, never on M, N or the launch grid.
 //
-// Memory: one warp per weight row.  Each warp streams its row (and, when the
-// row pitch allows, the row's scales) into its own shared-memory slot with a
-// single bulk copy issued at kernel start, so the whole weight is in flight
-// at once without holding registers.  Meanwhile the CTA requantises the
-// activation rows into shared memory (same rule and code as requant_a, so
-// the codes match it bit for bit), then each warp waits for its row and
-// forms the block dot products from shared memory.
+// Memory: one warp per weight row.  Lane 0 of each warp streams its row
+// (and, when the row pitch allows, the row's scales) into the warp's own
+// shared-memory slot as 1 KB bulk copies, each completing on its own
+// mbarrier, all issued at kernel start: the whole weight is in flight at
+// once without holding registers, and a warp consumes its first chunks while
+// the rest still stream.  Meanwhile the CTA requantises the activation rows
+// into shared memory (same rule and code as requant_a, so the codes match it
+// bit for bit).  Launched with programmatic dependent launch: activations
+// are read after waiting for the previous kernel on the stream; with the
+// static-weight option the first row's copies go out before that wait.  The
+// weight is one [N, K] tensor or a table of stacked segments.
 #include <cuda_bf16.h>
 
 #include "common.cuh"

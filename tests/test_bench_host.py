@@ -89,3 +89,21 @@ def test_stored_traffic_requires_matching_source(tmp_path, monkeypatch):
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: src)
     assert bench.stored_traffic("decode_kernel", "decode") == 123.0
     assert bench.stored_traffic("gemm_kernel", "decode") is None
+
+
+def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    import shutil
+
+    import bench
+
+    src = os.path.join(bench.ROOT, "block_scaled_precision_requant_b200", "csrc")
+    root = tmp_path / "r"
+    shutil.copytree(src, root / "block_scaled_precision_requant_b200" / "csrc")
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    h0 = bench.kernel_source_hash()
+    f = root / "block_scaled_precision_requant_b200" / "csrc" / "decode.cu"
+    text = f.read_text()
+    f.write_text("// a new comment line\n/* and a block\n   comment */\n" + text.replace("\n\n", "\n\n\n", 3))
+    assert bench.kernel_source_hash() == h0
+    f.write_text(text.replace("return MR <= 2 ? 32 : 8;", "return MR <= 2 ? 32 : 16;"))
+    assert bench.kernel_source_hash() != h0
