@@ -17,7 +17,10 @@ Sources (the launcher pages of the ``metrale_model_layers`` ops crate):
   writes BF16 ``out[M, N]``.  ``faith2_kernel`` takes no ``scale2`` argument,
   so ``scale2`` is folded into ``W_scale`` by the weight requantisation.
 * ``w4a4_proj/fixed.rs`` -- doc comment of ``nvfp4_proj_mx``: a row's output
-  bits do not depend on the row count or on the other rows.
+  bits do not depend on the row count or on the other rows; the same page's
+  W4A4 projection (a per-row NVFP4 quantiser of the BF16 input, then the
+  "mx" GEMV on the NVFP4 weight; its arithmetic is this module's reading,
+  see ``quantize_nvfp4_rows`` and ``w4a4_proj``).
 * ``w8a8_decode/parts.rs`` -- doc comment of ``W8a8Weight::segment``: a
   segment of a stacked weight yields the bits the stacked launch yields for
   those rows; ``W8a8Kernels::quant_silu``: the SiLU.mul quantiser (its
@@ -70,6 +73,10 @@ __all__ = [
     "silu_mul_bf16",
     "requant_silu_a",
     "w4a16_gemv",
+    "e4m3_encode_rne",
+    "e2m1_encode_rne",
+    "quantize_nvfp4_rows",
+    "w4a4_proj",
 ]
 
 GROUP = 32  # elements per int8 scale group
@@ -334,3 +341,97 @@ def w4a16_gemv(a_bits, w_packed, w_e4m3, scale2, k: int) -> np.ndarray:
     v = dequant_nvfp4(w_packed, w_e4m3, scale2, k).astype(np.float64)
     x = bf16_bits_to_f32(np.atleast_2d(np.asarray(a_bits, dtype=np.uint16))).astype(np.float64)
     return bf16_rne((x @ v.T).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
+# W4A4: NVFP4 activations (w4a4_proj/fixed.rs, `nvfp4_proj_mx`: a per-row
+# NVFP4 quantiser of the BF16 input, then the "mx" GEMV on the NVFP4 weight;
+# "the quantizer is per row, so a row's output bits do not depend on m or on
+# the other rows").  The page gives no arithmetic.  Readings taken
+# (provisional, for a later kernel):
+#   * the quantiser encodes each row as the weight is stored: per-row F32
+#     scale2 = RN(amax_row / 2688) (2688 = 6 * 448), per-16 E4M3 scale
+#     s16 = E4M3_RNE(RN(amax16 / RN(6 * scale2))), codes
+#     E2M1_RNE(RN(x / RN(s16 * scale2))); an all-zero row (or block) gets
+#     scale 0 and codes 0;
+#   * the product is the dot product of the dequantised operands,
+#     scale2_a * scale2_w * sum_k (e2m1_a * s16_a) * (e2m1_w * s16_w), in
+#     float64 (each term is exact there) and rounded to BF16 at the end; a GPU
+#     sums in float32 and is compared within the BF16 tolerance.
+# ---------------------------------------------------------------------------
+
+def _e4m3_table():
+    """All non-negative finite E4M3 values with their byte codes (0x00..0x7E)."""
+    codes = np.arange(0x7F, dtype=np.uint8)
+    return codes, e4m3_decode(codes).astype(np.float64)
+
+
+def e4m3_encode_rne(x) -> np.ndarray:
+    """Nearest E4M3 byte of non-negative x (ties to the even mantissa, i.e.
+    the even code; values above 448 saturate to 448), by search over the
+    table of all finite values."""
+    x = np.asarray(x, dtype=np.float64)
+    codes, vals = _e4m3_table()
+    d = np.abs(x[..., None] - vals)
+    best = d.min(axis=-1, keepdims=True)
+    tie_ok = d == best
+    # among equally near values prefer the even code (even mantissa)
+    pref = np.where(tie_ok & ((codes & 1) == 0), 0, np.where(tie_ok, 1, 2))
+    return codes[np.argmin(pref, axis=-1)].astype(np.uint8)
+
+
+def e2m1_encode_rne(y) -> np.ndarray:
+    """E2M1 nibble of y (sign of y in bit 3; magnitude rounded to the nearest
+    of {0, .5, 1, 1.5, 2, 3, 4, 6}, ties to the even mantissa, saturating at
+    6), by search over the table."""
+    y = np.asarray(y, dtype=np.float64)
+    mags = E2M1_MAGNITUDES.astype(np.float64)
+    d = np.abs(np.abs(y)[..., None] - mags)
+    best = d.min(axis=-1, keepdims=True)
+    tie_ok = d == best
+    idx = np.arange(8)
+    pref = np.where(tie_ok & ((idx & 1) == 0), 0, np.where(tie_ok, 1, 2))
+    mag = np.argmin(pref, axis=-1).astype(np.uint8)
+    sign = np.signbit(y).astype(np.uint8) << 3  # a negative value rounded to 0 is -0 (0x8)
+    return (mag | sign).astype(np.uint8)
+
+
+def quantize_nvfp4_rows(a_bits: np.ndarray):
+    """The per-row NVFP4 quantiser of BF16 rows [M, K] (K % 16 == 0):
+    (packed codes u8 [M, K/2], E4M3 bytes u8 [M, K/16], scale2 f32 [M])."""
+    x = bf16_bits_to_f32(np.atleast_2d(np.asarray(a_bits, dtype=np.uint16)))
+    m, k = x.shape
+    f32 = np.float32
+    amax = np.max(np.abs(x), axis=1)
+    scale2 = (amax / f32(2688.0)).astype(np.float32)
+    blocks = x.reshape(m, k // 16, 16)
+    amax16 = np.max(np.abs(blocks), axis=2)
+    six_s2 = (f32(6.0) * scale2).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        t = np.where(six_s2[:, None] > 0, (amax16 / six_s2[:, None]).astype(np.float32), f32(0.0))
+    e4 = e4m3_encode_rne(t)
+    s16 = e4m3_decode(e4)
+    denom = (s16 * scale2[:, None]).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        y = np.where(denom[..., None] > 0, (blocks / denom[..., None]).astype(np.float32), f32(0.0))
+    codes = e2m1_encode_rne(y).reshape(m, k)
+    packed = ((codes[:, 0::2] & 0xF) | ((codes[:, 1::2] & 0xF) << 4)).astype(np.uint8)
+    return packed, e4.astype(np.uint8), scale2
+
+
+def _nvfp4_unscaled(packed, e4, k: int) -> np.ndarray:
+    """e2m1(c) * e4m3(s16) per element, float64 (exact), without scale2."""
+    codes = unpack_nvfp4(packed, k)
+    n = codes.shape[0]
+    s16 = np.repeat(e4m3_decode(np.asarray(e4).reshape(n, k // 16)), 16, axis=1)
+    return e2m1_decode(codes).astype(np.float64) * s16.astype(np.float64)
+
+
+def w4a4_proj(a_bits, w_packed, w_e4m3, scale2_w, k: int) -> np.ndarray:
+    """BF16 output bits [M, N] of the W4A4 projection: the row quantiser
+    above, then the dequantised dot product (float64) times both F32 scales."""
+    ap, ae, as2 = quantize_nvfp4_rows(a_bits)
+    va = _nvfp4_unscaled(ap, ae, k)
+    vw = _nvfp4_unscaled(w_packed, w_e4m3, k)
+    acc = (va @ vw.T) * (as2.astype(np.float64)[:, None] * float(np.float32(scale2_w)))
+    return bf16_rne(acc.astype(np.float32))
