@@ -213,12 +213,41 @@ def roofline(bound, achieved, peak, unit, traffic):
             "frac": (achieved / peak) if peak else None, "traffic": traffic}
 
 
-def kernel_source_hash():
-    """Hash of the CUDA sources with comments and whitespace removed: stored
-    ncu traffic counts are valid only for this code."""
+# translation unit of each measured kernel; with the csrc headers it includes
+# and the C-ABI layer that picks its launch parameters, these are the sources
+# its DRAM traffic depends on
+KERNEL_UNITS = {"decode_kernel": "decode.cu", "gemm_kernel": "gemm_tc.cu"}
+LAUNCH_LAYER = "api.cu"
+
+
+def _csrc_dir():
+    return os.path.join(ROOT, "block_scaled_precision_requant_b200", "csrc")
+
+
+def kernel_sources(kernel: str):
+    """Sorted csrc file names that the kernel's code and launch depend on:
+    its translation unit, the launch layer, and every csrc header they
+    include, transitively."""
+    csrc = _csrc_dir()
+    todo = [KERNEL_UNITS[kernel], LAUNCH_LAYER]
+    seen = set()
+    while todo:
+        name = todo.pop()
+        if name in seen or not os.path.exists(os.path.join(csrc, name)):
+            continue
+        seen.add(name)
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            todo += re.findall(r'^\s*#\s*include\s+"([^"]+)"', f.read(), flags=re.M)
+    return sorted(seen)
+
+
+def kernel_source_hash(kernel: str):
+    """Hash of the kernel's sources (kernel_sources) with comments and
+    whitespace removed: stored ncu traffic counts are valid only for this
+    code.  Files the kernel does not depend on do not enter it."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "block_scaled_precision_requant_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    csrc = _csrc_dir()
+    for name in kernel_sources(kernel):
         with open(os.path.join(csrc, name), encoding="utf-8") as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)  # block comments
@@ -238,7 +267,7 @@ def stored_traffic(kernel: str, workload: str):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel) if kernel in KERNEL_UNITS else None
     for line in lines:
         parts = line.split()
         if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[2] == src:

@@ -83,27 +83,50 @@ def test_units_and_bytes():
 def test_stored_traffic_requires_matching_source(tmp_path, monkeypatch):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    src = bench.kernel_source_hash()
+    src = bench.kernel_source_hash("decode_kernel")
     (prof / "dram_traffic.txt").write_text(f"decode_kernel decode {src} 123\ndecode_kernel decode deadbeef 7\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: src)
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda kernel: src)
     assert bench.stored_traffic("decode_kernel", "decode") == 123.0
     assert bench.stored_traffic("gemm_kernel", "decode") is None
+    assert bench.stored_traffic("no_such_kernel", "decode") is None
 
 
-def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+def _csrc_copy(tmp_path, monkeypatch):
     import shutil
-
-    import bench
 
     src = os.path.join(bench.ROOT, "block_scaled_precision_requant_b200", "csrc")
     root = tmp_path / "r"
-    shutil.copytree(src, root / "block_scaled_precision_requant_b200" / "csrc")
+    csrc = root / "block_scaled_precision_requant_b200" / "csrc"
+    shutil.copytree(src, csrc)
     monkeypatch.setattr(bench, "ROOT", str(root))
-    h0 = bench.kernel_source_hash()
-    f = root / "block_scaled_precision_requant_b200" / "csrc" / "decode.cu"
+    return csrc
+
+
+def test_source_hash_ignores_comments_not_code(tmp_path, monkeypatch):
+    csrc = _csrc_copy(tmp_path, monkeypatch)
+    h0 = bench.kernel_source_hash("decode_kernel")
+    f = csrc / "decode.cu"
     text = f.read_text()
     f.write_text("// a new comment line\n/* and a block\n   comment */\n" + text.replace("\n\n", "\n\n\n", 3))
-    assert bench.kernel_source_hash() == h0
+    assert bench.kernel_source_hash("decode_kernel") == h0
     f.write_text(text.replace("return MR <= 2 ? 32 : 8;", "return MR <= 2 ? 32 : 16;"))
-    assert bench.kernel_source_hash() != h0
+    assert bench.kernel_source_hash("decode_kernel") != h0
+
+
+def test_source_hash_follows_the_kernels_own_sources(tmp_path, monkeypatch):
+    csrc = _csrc_copy(tmp_path, monkeypatch)
+    assert bench.kernel_sources("decode_kernel") == ["api.cu", "common.cuh", "decode.cu", "kernels.h", "quant.cuh"]
+    assert bench.kernel_sources("gemm_kernel") == ["api.cu", "common.cuh", "gemm_tc.cu", "kernels.h"]
+    h = {k: bench.kernel_source_hash(k) for k in bench.KERNEL_UNITS}
+    # a new, unrelated translation unit changes neither
+    (csrc / "other.cu").write_text("__global__ void other_kernel() {}\n")
+    assert {k: bench.kernel_source_hash(k) for k in bench.KERNEL_UNITS} == h
+    # a shared header changes both; a kernel's own unit changes only it
+    (csrc / "common.cuh").write_text((csrc / "common.cuh").read_text() + "\nconstexpr int kProbe = 1;\n")
+    h2 = {k: bench.kernel_source_hash(k) for k in bench.KERNEL_UNITS}
+    assert all(h2[k] != h[k] for k in h)
+    (csrc / "gemm_tc.cu").write_text((csrc / "gemm_tc.cu").read_text() + "\nstatic int probe_value = 2;\n")
+    assert bench.kernel_source_hash("gemm_kernel") != h2["gemm_kernel"]
+    assert bench.kernel_source_hash("decode_kernel") == h2["decode_kernel"]
+
