@@ -370,7 +370,7 @@ def e4m3_encode_rne(x) -> np.ndarray:
     """Nearest E4M3 byte of non-negative x (ties to the even mantissa, i.e.
     the even code; values above 448 saturate to 448), by search over the
     table of all finite values."""
-    x = np.asarray(x, dtype=np.float64)
+    x = np.minimum(np.asarray(x, dtype=np.float64), 448.0)  # saturation first: no ties among huge distances
     codes, vals = _e4m3_table()
     d = np.abs(x[..., None] - vals)
     best = d.min(axis=-1, keepdims=True)
@@ -386,7 +386,7 @@ def e2m1_encode_rne(y) -> np.ndarray:
     6), by search over the table."""
     y = np.asarray(y, dtype=np.float64)
     mags = E2M1_MAGNITUDES.astype(np.float64)
-    d = np.abs(np.abs(y)[..., None] - mags)
+    d = np.abs(np.minimum(np.abs(y), 6.0)[..., None] - mags)  # saturation first, as for E4M3
     best = d.min(axis=-1, keepdims=True)
     tie_ok = d == best
     idx = np.arange(8)

@@ -53,14 +53,14 @@ def test_e4m3_encoder_matches_torch_cast():
 
 
 def test_e4m3_encoder_saturates():
-    assert np.all(oracle.e4m3_encode_rne(np.array([448.0, 464.0, 470.0, 1e6])) == 0x7E)
+    assert np.all(oracle.e4m3_encode_rne(np.array([448.0, 464.0, 470.0, 1e6, 1e30, np.inf])) == 0x7E)
 
 
 def test_e2m1_encoder_by_hand():
     ys = {
         0.0: 0, 0.24: 0, 0.25: 0, 0.26: 1, 0.5: 1, 0.75: 2, 1.0: 2, 1.25: 2, 1.26: 3,
         1.5: 3, 1.75: 4, 2.0: 4, 2.5: 4, 2.51: 5, 3.0: 5, 3.5: 6, 4.0: 6, 4.99: 6,
-        5.0: 6, 5.01: 7, 6.0: 7, 7.0: 7, 1e9: 7,
+        5.0: 6, 5.01: 7, 6.0: 7, 7.0: 7, 1e9: 7, 1e30: 7, float("inf"): 7,
     }
     y = np.array(list(ys), dtype=np.float32)
     want = np.array(list(ys.values()), dtype=np.uint8)
