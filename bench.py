@@ -712,6 +712,54 @@ def oracle_seconds(fn, budget_s, max_calls=50):
     return spent / done, done
 
 
+def w4a4_extra(device, wl, host, steps, cpu=True):
+    """The NVFP4 W4A4 decode GEMV (activation rows quantised to NVFP4 inside
+    the kernel) on the decode workload's weight as stored: a CUDA-graph loop
+    over rotating copies (>= 3x L2), bytes = N*K*0.5625 + 2MK + 2MN per step."""
+    import torch
+
+    import block_scaled_precision_requant_b200 as bsr
+
+    m, n, k = wl.shape
+    nbytes = n * k // 2 + n * k // 16 + 2 * m * k + 2 * m * n
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    copies = max(2, -(-3 * l2 // nbytes))
+    wp = torch.from_numpy(host["w_packed"]).to(device)
+    we = torch.from_numpy(host["w_e4m3"]).to(device)
+    a = torch.from_numpy(host["a_bits"].view(np.int16)).view(torch.bfloat16).to(device)
+    ws = [(wp.clone(), we.clone()) for _ in range(copies)]
+    s2 = float(host["scale2"])
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    for i in range(3):
+        bsr.w4a4_decode(a, *ws[i % copies], s2, out)
+    torch.cuda.synchronize()
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for i in range(steps):
+            bsr.w4a4_decode(a, *ws[i % copies], s2, out)
+    gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    del gr, ws
+    if bsr.device_status() != 0:
+        raise RuntimeError(f"device status word {bsr.device_status()}")
+    res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
+           "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
+    if cpu:
+        import oracle
+
+        t, calls = oracle_seconds(lambda: oracle.w4a4_proj(host["a_bits"], host["w_packed"], host["w_e4m3"],
+                                                           host["scale2"], k), 3.0)
+        res["cpu_baseline"] = {"kind": "oracle", "cores": 1, "gbs": nbytes / t / 1e9, "ms_per_step": t * 1e3,
+                               "sample": f"{calls} full step(s) (M={m})"}
+    return res
+
+
 def stacked_prefill_extra(device, steps, warmup):
     """Prefill over a stacked weight shaped like Q, K and V of a grouped-query
     layer (4096 + 1024 + 1024 rows, K = 4096, M = 2048): bsr_proj_stacked
@@ -880,6 +928,7 @@ def gpu_main(args):
         "requant_w": {"gbs": n * k * 1.6875 / (ms_rw / 1e3) / 1e9, "ms": ms_rw,
                       "frac_of_hbm": n * k * 1.6875 / (ms_rw / 1e3) / 1e9 / peaks["hbm_gbs"]},
     }
+    host = g.host
     del g
     torch.cuda.empty_cache()
     if not args.no_extra and world == 1:
@@ -894,6 +943,10 @@ def gpu_main(args):
         line["stacked_prefill"] = stacked_prefill_extra(dev, min(args.steps, 10), 3)
         if decode:
             line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks, cpu=not args.no_cpu)
+            try:  # the last GPU work of the run: an error here costs only this entry
+                line["w4a4_decode"] = w4a4_extra(dev, wl, host, max(args.steps, 20), cpu=not args.no_cpu)
+            except Exception as exc:  # noqa: BLE001 - reported in the line
+                line["w4a4_decode"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_seconds)
     if rank == 0:

@@ -50,6 +50,8 @@ __all__ = [
     "decode_stacked",
     "proj_stacked",
     "w4a16_decode",
+    "quant_nvfp4_rows",
+    "w4a4_decode",
     "silu_mul",
     "requant_silu_a",
     "proj_silu_scratch_bytes",
@@ -95,6 +97,8 @@ SIGNATURES = [
     ("bsr_decode_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_proj_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_w4a16_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
+    ("bsr_nvfp4_quant_rows", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
+    ("bsr_w4a4_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
     ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
@@ -506,6 +510,53 @@ def w4a16_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
         out = _empty((m, n), torch.bfloat16, a)
     _check(
         lib().bsr_w4a16_decode(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(w_packed, torch.uint8, (n, k // 2), "w_packed"),
+            _dev(w_e4m3, torch.uint8, (n, k // 16), "w_e4m3"),
+            ctypes.c_float(float(scale2)),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def quant_nvfp4_rows(a, out=None, stream=None):
+    """Per-row NVFP4 quantiser of the W4A4 path: a [M, K] bfloat16 ->
+    (a_packed [M, K/2] uint8, a_e4m3 [M, K/16] uint8, a_scale2 [M] float32)."""
+    torch = _torch()
+    m, k = a.shape
+    if out is None:
+        out = (_empty((m, k // 2), torch.uint8, a), _empty((m, k // 16), torch.uint8, a),
+               _empty((m,), torch.float32, a))
+    packed, e4, s2 = out
+    _check(
+        lib().bsr_nvfp4_quant_rows(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(packed, torch.uint8, (m, k // 2), "a_packed"),
+            _dev(e4, torch.uint8, (m, k // 16), "a_e4m3"),
+            _dev(s2, torch.float32, (m,), "a_scale2"),
+            m,
+            k,
+            _stream_ptr(stream),
+        )
+    )
+    return packed, e4, s2
+
+
+def w4a4_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
+    """NVFP4 W4A4 decode GEMV (activation rows quantised to NVFP4 inside the
+    kernel) -> out [M, N] bfloat16."""
+    torch = _torch()
+    m, k = a.shape
+    n = w_packed.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    _check(
+        lib().bsr_w4a4_decode(
             _dev(a, torch.bfloat16, (m, k), "a"),
             _dev(w_packed, torch.uint8, (n, k // 2), "w_packed"),
             _dev(w_e4m3, torch.uint8, (n, k // 16), "w_e4m3"),

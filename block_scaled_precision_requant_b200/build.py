@@ -18,8 +18,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbsr.so")
-SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "w4a16.cu"]
-HEADERS = ["common.cuh", "quant.cuh", "kernels.h"]
+SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "w4a16.cu",
+           "w4a4.cu"]
+HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -225,6 +225,38 @@ bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const ui
                             uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
 
 /*
+ * NVFP4 W4A4 (w4a4_proj/fixed.rs, `nvfp4_proj_mx`: a per-row NVFP4 quantiser
+ * of the BF16 input, then the "mx" GEMV on the NVFP4 weight; a row's output
+ * bits do not depend on M or on the other rows).  The page gives no
+ * arithmetic; reading taken: each activation row is encoded the way the
+ * weight is stored,
+ *   scale2 = RN(amax_row / 2688),  s16 = E4M3_RNE(RN(amax16 / RN(6 * scale2))),
+ *   code = E2M1_RNE(RN(x / RN(s16 * scale2)))
+ * (float32 operations rounded to nearest; E4M3 saturating at 448, E2M1 at 6
+ * with ties to the even mantissa and the sign kept; a zero row or block gets
+ * scale 0 and codes 0), and the product is
+ *   out[m, n] = bf16( scale2_a[m] * scale2_w * sum_b s16a * s16w * sum_16 ea * ew ).
+ * K > 0, K % 16 == 0; pointers 16-byte aligned (out 2-byte).  Inputs finite.
+ */
+
+/* The row quantiser alone: a [M, K] BF16 in; a_packed [M, K/2] (element 2i in
+ * the low nibble of byte i), a_e4m3 [M, K/16] and a_scale2 [M] float out,
+ * bit-exact with the CPU oracle. */
+bsr_status bsr_nvfp4_quant_rows(const uint16_t* a, uint8_t* a_packed, uint8_t* a_e4m3, float* a_scale2, int64_t m,
+                                int64_t k, void* stream);
+
+/* The W4A4 decode GEMV, the quantiser fused in (each CTA quantises its rows
+ * of A into shared memory): a [M, K] BF16, w_packed [N, K/2], w_e4m3
+ * [N, K/16], scale2 the weight's F32 scale (host value), out [M, N] BF16.
+ * The products of a 16-block are exact, the sum over blocks is float32:
+ * results agree with the exact product within the BF16 tolerance, and a
+ * row's bits do not depend on M or on the other rows.  Any M (built for
+ * M <= 16); the quantised rows of up to 16 rows, K * 0.5625 + 4 bytes
+ * each, must fit in the device's shared memory per CTA (BSR_ESHAPE). */
+bsr_status bsr_w4a4_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                           uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
+
+/*
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
  * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:
  *   x = bf16_rne(silu(g) * u),  silu(g) = g / (1 + exp(-g)),

@@ -97,6 +97,23 @@ def test_stacked_argument_errors(L):
     assert L.bsr_decode_stacked(_fake(256), arr, arr, n1, 1, _fake(256), 1, 64, 4, None) == 1
 
 
+def test_w4a4_argument_errors(L):
+    f = ctypes.c_float(1.0)
+    assert L.bsr_w4a4_decode(_fake(256), _fake(256), _fake(256), f, _fake(256), 1, 8, 40, None) == 3
+    assert "multiple of 16" in bsr.last_error()
+    assert L.bsr_w4a4_decode(_fake(256), _fake(256), _fake(256), f, _fake(256), 1, 8, 0, None) == 3
+    assert L.bsr_w4a4_decode(_fake(256), _fake(256), _fake(256), f, _fake(256), 1, -1, 48, None) == 1
+    assert L.bsr_w4a4_decode(None, _fake(256), _fake(256), f, _fake(256), 1, 8, 48, None) == 1
+    assert L.bsr_w4a4_decode(_fake(264), _fake(256), _fake(256), f, _fake(256), 1, 8, 48, None) == 2
+    assert L.bsr_w4a4_decode(_fake(256), _fake(256), _fake(256), f, _fake(257), 1, 8, 48, None) == 2
+    assert L.bsr_w4a4_decode(None, None, None, f, None, 0, 8, 48, None) == 0
+    assert L.bsr_w4a4_decode(None, None, None, f, None, 3, 0, 48, None) == 0
+    assert L.bsr_nvfp4_quant_rows(_fake(256), _fake(256), _fake(256), _fake(256), 2, 24, None) == 3
+    assert L.bsr_nvfp4_quant_rows(_fake(256), _fake(256), _fake(256), _fake(260), 2, 32, None) == 2
+    assert L.bsr_nvfp4_quant_rows(_fake(256), None, _fake(256), _fake(256), 2, 32, None) == 1
+    assert L.bsr_nvfp4_quant_rows(None, None, None, None, 0, 32, None) == 0
+
+
 def test_scratch_errors(L):
     m, k = 64, 256
     need = L.bsr_proj_scratch_bytes(m, k)
