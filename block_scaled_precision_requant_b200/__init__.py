@@ -52,6 +52,9 @@ __all__ = [
     "w4a16_decode",
     "quant_nvfp4_rows",
     "w4a4_decode",
+    "sf_blocked_bytes",
+    "sf_blocked",
+    "w4a4_gemm",
     "silu_mul",
     "requant_silu_a",
     "proj_silu_scratch_bytes",
@@ -99,6 +102,9 @@ SIGNATURES = [
     ("bsr_w4a16_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
     ("bsr_nvfp4_quant_rows", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_w4a4_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
+    ("bsr_nvfp4_sf_blocked_bytes", ctypes.c_size_t, [_I64, _I64]),
+    ("bsr_nvfp4_sf_blocked", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
+    ("bsr_w4a4_gemm", ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P, _P]),
     ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
@@ -565,6 +571,61 @@ def w4a4_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
             m,
             n,
             k,
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def sf_blocked_bytes(rows: int, k: int) -> int:
+    """Bytes of the blocked scale layout of the W4A4 GEMM (0 if invalid)."""
+    return int(lib().bsr_nvfp4_sf_blocked_bytes(rows, k))
+
+
+def sf_blocked(e4m3, out=None, stream=None):
+    """Row-major E4M3 scales [rows, K/16] uint8 -> the W4A4 GEMM's blocked
+    layout (uint8 [sf_blocked_bytes(rows, K)])."""
+    torch = _torch()
+    rows, kb = e4m3.shape
+    k = kb * 16
+    nbytes = sf_blocked_bytes(rows, k)
+    if out is None:
+        out = _empty((nbytes,), torch.uint8, e4m3)
+    _check(
+        lib().bsr_nvfp4_sf_blocked(
+            _dev(e4m3, torch.uint8, (rows, kb), "e4m3"), _dev(out, torch.uint8, (nbytes,), "blocked"), rows, k,
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def w4a4_gemm(a_packed, a_sf_blocked, a_scale2, w_packed, w_sf_blocked, scale2: float, out=None, status=None,
+              stream=None):
+    """W4A4 GEMM on the tensor cores -> out [M, N] bfloat16.  `status` is a
+    device int32 tensor of one element into which a timed-out wait ORs its
+    bit (a fresh zero one when omitted)."""
+    torch = _torch()
+    m, kh = a_packed.shape
+    n = w_packed.shape[0]
+    k = 2 * kh
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a_packed)
+    if status is None:
+        status = torch.zeros((1,), dtype=torch.int32, device=a_packed.device)
+    _check(
+        lib().bsr_w4a4_gemm(
+            _dev(a_packed, torch.uint8, (m, kh), "a_packed"),
+            _dev(a_sf_blocked, torch.uint8, (sf_blocked_bytes(m, k),), "a_sf_blocked"),
+            _dev(a_scale2, torch.float32, (m,), "a_scale2"),
+            _dev(w_packed, torch.uint8, (n, kh), "w_packed"),
+            _dev(w_sf_blocked, torch.uint8, (sf_blocked_bytes(n, k),), "w_sf_blocked"),
+            ctypes.c_float(float(scale2)),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            _dev(status, torch.int32, (1,), "status"),
             _stream_ptr(stream),
         )
     )

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbsr.so")
 SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "w4a16.cu",
-           "w4a4.cu"]
+           "w4a4.cu", "w4a4_gemm.cu"]
 HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh"]
 
 NVCC_FLAGS = [

@@ -257,6 +257,32 @@ bsr_status bsr_w4a4_decode(const uint16_t* a, const uint8_t* w_packed, const uin
                            uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
 
 /*
+ * W4A4 on the tensor cores (block-scaled FP4 MMA, kind::mxf4nvf4): the same
+ * product as bsr_w4a4_decode, accumulated in FP32 by the MMA.  The E4M3 scale
+ * bytes must be non-negative (sign bit clear) and are passed in a blocked
+ * layout: for 128-row tile t and K group g (64 elements) a 512-byte atom at
+ * offset (t * K/64 + g) * 512 whose 32-bit word 4*r0 + r1 holds the four
+ * scales of row 128t + r0 + 32*r1 (r0 < 32, r1 < 4), scale 4g + j in byte j;
+ * rows past the matrix are zero.
+ */
+
+/* Bytes of the blocked layout for `rows` rows: ceil(rows/128) * K/64 * 512
+ * (0 for invalid sizes; K % 64 == 0). */
+size_t bsr_nvfp4_sf_blocked_bytes(int64_t rows, int64_t k);
+
+/* Row-major E4M3 scales e4m3 [rows, K/16] -> blocked [bsr_nvfp4_sf_blocked_bytes]
+ * (once per weight; per call for activations).  16-byte aligned pointers. */
+bsr_status bsr_nvfp4_sf_blocked(const uint8_t* e4m3, uint8_t* blocked, int64_t rows, int64_t k, void* stream);
+
+/* out [M, N] BF16 = W4A4 product of a_packed [M, K/2] (scales a_sf_blocked,
+ * a_scale2 [M]) and w_packed [N, K/2] (scales w_sf_blocked, scale2 host
+ * value).  K % 256 == 0; every array 16-byte aligned.  status_dev: a
+ * caller-owned device int into which a wait that runs out ORs its bit. */
+bsr_status bsr_w4a4_gemm(const uint8_t* a_packed, const uint8_t* a_sf_blocked, const float* a_scale2,
+                         const uint8_t* w_packed, const uint8_t* w_sf_blocked, float scale2, uint16_t* out, int64_t m,
+                         int64_t n, int64_t k, int* status_dev, void* stream);
+
+/*
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
  * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:
  *   x = bf16_rne(silu(g) * u),  silu(g) = g / (1 + exp(-g)),

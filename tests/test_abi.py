@@ -114,6 +114,24 @@ def test_w4a4_argument_errors(L):
     assert L.bsr_nvfp4_quant_rows(None, None, None, None, 0, 32, None) == 0
 
 
+def test_w4a4_gemm_argument_errors(L):
+    f = ctypes.c_float(1.0)
+    assert L.bsr_nvfp4_sf_blocked_bytes(1, 64) == 512
+    assert L.bsr_nvfp4_sf_blocked_bytes(129, 256) == 2 * 4 * 512
+    assert L.bsr_nvfp4_sf_blocked_bytes(128, 96) == 0 and L.bsr_nvfp4_sf_blocked_bytes(0, 64) == 0
+    assert L.bsr_nvfp4_sf_blocked(_fake(256), _fake(256), 4, 96, None) == 3
+    assert L.bsr_nvfp4_sf_blocked(_fake(256), _fake(264), 4, 64, None) == 2
+    assert L.bsr_nvfp4_sf_blocked(None, _fake(256), 4, 64, None) == 1
+    assert L.bsr_nvfp4_sf_blocked(None, None, 0, 64, None) == 0
+    args = [_fake(256)] * 5
+    assert L.bsr_w4a4_gemm(*args, f, _fake(256), 4, 8, 128, _fake(256), None) == 3
+    assert "multiple of 256" in bsr.last_error()
+    assert L.bsr_w4a4_gemm(*args, f, _fake(256), 4, -8, 256, _fake(256), None) == 1
+    assert L.bsr_w4a4_gemm(*args, f, _fake(256), 4, 8, 256, None, None) == 1
+    assert L.bsr_w4a4_gemm(*args[:4], _fake(264), f, _fake(256), 4, 8, 256, _fake(256), None) == 2
+    assert L.bsr_w4a4_gemm(None, None, None, None, None, f, None, 0, 8, 256, None, None) == 0
+
+
 def test_scratch_errors(L):
     m, k = 64, 256
     need = L.bsr_proj_scratch_bytes(m, k)

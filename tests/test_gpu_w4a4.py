@@ -8,6 +8,8 @@
   oracle.w4a4_proj (exact sums) for M = 1 at the decode size, every M up to
   16 and beyond, ragged N, K % 256 != 0 and K = 16; a row's bits do not
   depend on M or on the other rows; an all-zero row gives +0 bits.
+* The relayout of row-major E4M3 scales into the tensor-core GEMM's blocked
+  layout, byte for byte against the layout restated in numpy.
 """
 import numpy as np
 import pytest
@@ -89,3 +91,28 @@ def test_w4a4_row_invariance_and_zero_row():
     assert np.all(got[zr] == 0)
     ref = oracle.w4a4_proj(a_bits, w["w_packed"], w["w_e4m3"], w["scale2"], k)
     assert_close_bf16(got, ref, "w4a4 laplace rows")
+
+
+def _blocked_reference(e4, rows, k):
+    """The blocked scale layout restated in numpy: atom (t, g) at
+    (t * K/64 + g) * 512, word 4*r0 + r1 = the four scales 4g..4g+3 of row
+    128t + r0 + 32*r1, zero past the last row."""
+    tiles, groups = -(-rows // 128), k // 64
+    out = np.zeros((tiles, groups, 32, 4, 4), dtype=np.uint8)  # [t][g][r0][r1][byte]
+    for t in range(tiles):
+        for r1 in range(4):
+            for r0 in range(32):
+                row = 128 * t + r0 + 32 * r1
+                if row < rows:
+                    out[t, :, r0, r1, :] = e4[row].reshape(groups, 4)
+    return out.reshape(-1)
+
+
+@pytest.mark.parametrize("rows,k", [(1, 64), (130, 256), (300, 1024)])
+def test_scale_relayout_to_blocked(rows, k):
+    rng = np.random.default_rng(rows + k)
+    e4 = rng.integers(0, 0x7F, size=(rows, k // 16), dtype=np.uint8)
+    got = bsr.sf_blocked(up_u8(e4))
+    torch.cuda.synchronize()
+    assert got.numel() == bsr.sf_blocked_bytes(rows, k)
+    assert np.array_equal(got.cpu().numpy(), _blocked_reference(e4, rows, k))
