@@ -21,6 +21,8 @@
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -152,14 +154,18 @@ cudaError_t launch_w4a16_t(const uint16_t* a, const uint8_t* w_packed, const uin
   const size_t smem = (size_t)MR * (size_t)k * 2;
   if (smem > smem_limit) return cudaErrorInvalidValue;
   static size_t granted[64] = {};
+  static std::mutex mu;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem > granted[dev] && smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    granted[dev] = smem;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (smem > granted[dev] && smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      granted[dev] = smem;
+    }
   }
   // warps (= weight rows in flight) per CTA: spread the rows over all SMs
   int w = (int)((n + (long long)num_sms - 1) / num_sms);
