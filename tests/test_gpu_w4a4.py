@@ -3,7 +3,8 @@
 * The row quantiser: codes, E4M3 scales and F32 row scales bit-exact with
   oracle.quantize_nvfp4_rows on ragged shapes, rows whose float32 quotients
   land on E2M1 / E4M3 midpoints, zero rows and blocks, -0 entries, subnormal
-  rows and rows near the BF16 maximum.
+  rows and rows near the BF16 maximum, and equal to the hand-derived rows of
+  tests/golden/w4a4_rows.txt.
 * The decode GEMV: BF16 outputs within the projection tolerance of
   oracle.w4a4_proj (exact sums) for M = 1 at the decode size, every M up to
   16 and beyond, ragged N, K % 256 != 0 and K = 16; a row's bits do not
@@ -57,6 +58,16 @@ def test_quantiser_special_rows():
     a = _bf16(np.stack(rows))
     a[5, ::7] = 0x8000  # -0 inside non-zero blocks
     _check_quant(a)
+
+
+def test_quantiser_hand_derived_rows():
+    from tests.test_oracle_w4a4 import golden_rows
+
+    for name, bits, s2, e4, codes in golden_rows():
+        p, e, s = bsr.quant_nvfp4_rows(up_bf16(bits))
+        torch.cuda.synchronize()
+        assert f32(s)[0] == s2 and np.array_equal(e.cpu().numpy()[0], e4), name
+        assert np.array_equal(oracle.unpack_nvfp4(p.cpu().numpy(), bits.shape[1])[0], codes), name
 
 
 def _run(m, n, k, seed, recipe="normal_outlier_channels"):

@@ -9,7 +9,8 @@ host with g++, against the CPU oracle and PyTorch -- no GPU needed:
 * the row quantiser (same order as the kernels) against
   oracle.quantize_nvfp4_rows bit for bit: random rows with outlier channels,
   a zero row, -0 entries, rows whose float32 quotients land on midpoints,
-  subnormal BF16 rows (scale2 subnormal), and rows near the BF16 maximum.
+  subnormal BF16 rows (scale2 subnormal), rows near the BF16 maximum, and
+  the hand-derived rows of tests/golden/w4a4_rows.txt.
 """
 import ctypes
 import os
@@ -150,3 +151,12 @@ def test_row_quantiser_on_float32_midpoints(lib):
     for seed in (3, 10):
         a, _ = synth.make_activations(32, 1024, seed, "normal_outlier_channels")
         _assert_rows_equal(lib, a)
+
+
+def test_row_quantiser_hand_derived_rows(lib):
+    from tests.test_oracle_w4a4 import golden_rows
+
+    for name, bits, s2, e4, codes in golden_rows():
+        p, e, s = _quant_rows(lib, bits)
+        assert s[0] == s2 and np.array_equal(e[0], e4), name
+        assert np.array_equal(oracle.unpack_nvfp4(p, bits.shape[1])[0], codes), name

@@ -6,6 +6,9 @@ quantize_nvfp4_rows, w4a4_proj) against things other than the oracle:
   midpoint, and points just beside each midpoint; saturation above 448;
 * the E2M1 encoder on its midpoints and neighbours, worked out by hand from
   the grid {0, .5, 1, 1.5, 2, 3, 4, 6};
+* whole rows derived by hand (tests/golden/w4a4_rows.txt): an exact ladder,
+  a rounded E4M3 scale, saturation, every E2M1 midpoint, an E4M3 midpoint,
+  zero and negative-zero rows;
 * the row quantiser against the weight generator's encoder (an independent
   implementation: thresholds and float64 intermediates instead of table
   search and float32 steps) -- equal except where the float32 quotient lands
@@ -25,6 +28,7 @@ import torch
 
 import oracle
 from block_scaled_precision_requant_b200 import synth
+from tests import _golden
 
 F32 = np.float32
 
@@ -71,6 +75,29 @@ def test_e2m1_encoder_by_hand():
 # --------------------------------------------------------------------------
 # Row quantiser
 # --------------------------------------------------------------------------
+
+
+def golden_rows():
+    """(name, BF16 bits [1, K], scale2, e4m3 bytes, codes) of each hand-derived row."""
+    out = []
+    for c in _golden.cases("w4a4_rows.txt"):
+        x = np.array([float(v) for v in c["x"]], dtype=np.float32)
+        bits = oracle.bf16_rne(x)
+        # the fixture's decimals are exact in BF16, signs of zero included
+        assert np.array_equal(oracle.bf16_bits_to_f32(bits).view(np.uint32), x.view(np.uint32)), c["name"]
+        out.append((c["name"], bits[None], np.float32(c["scale2"][0]),
+                    np.array([int(v, 16) for v in c["e4m3"]], dtype=np.uint8),
+                    np.array([int(v, 16) for v in c["codes"]], dtype=np.uint8)))
+    return out
+
+
+def test_row_quantiser_hand_derived_rows():
+    for name, bits, s2, e4, codes in golden_rows():
+        k = bits.shape[1]
+        p, e, s = oracle.quantize_nvfp4_rows(bits)
+        assert s[0] == s2, name
+        assert np.array_equal(e[0], e4), name
+        assert np.array_equal(oracle.unpack_nvfp4(p, k)[0], codes), name
 
 
 def _rows(m, k, seed):
