@@ -287,6 +287,15 @@ def workload_desc(wl):
             "l2": "flushed before every timed step (256 MiB device write, outside the step events)"}
 
 
+def input_hashes(d):
+    """SHA-256 of every input buffer of a generated workload (the NVFP4
+    weight's nibbles and E4M3 bytes, its F32 scale2, the BF16 activations)."""
+    from block_scaled_precision_requant_b200 import synth
+
+    return {"w_packed": synth.sha256(d["w_packed"]), "w_e4m3": synth.sha256(d["w_e4m3"]),
+            "scale2": synth.sha256(np.asarray(d["scale2"], dtype=np.float32)), "a_bf16": synth.sha256(d["a_bits"])}
+
+
 def decode_bytes(m, n, k):
     """Algorithmic HBM bytes of one decode step: int8 weight, its F32 scales
     (4 B per 32), BF16 activations in, BF16 outputs out."""
@@ -489,6 +498,7 @@ class OracleRunner:
         self.w_i8, self.w_s = oracle.requant_w(d["w_packed"], d["w_e4m3"], d["scale2"], k)
         self.a = d["a_bits"]
         self.rows = synth.sample_rows(m, min(m, 64), self.wl.seed)
+        self.hashes = input_hashes(d)
 
     def sample_step(self, nrows):
         """Oracle projection of `nrows` sampled rows; returns seconds."""
@@ -540,7 +550,7 @@ def reference_main(args):
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded generator)", "impl": "reference",
-            "config": workload_desc(wl),
+            "config": {**workload_desc(wl), "inputs_sha256": r.hashes},
             "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
                              "sample": f"each step: the oracle on 1 of {len(r.rows)} sampled activation rows against the "
                                        f"full requantised weight; step time = per-row time x M={wl.m}"},
@@ -914,6 +924,7 @@ def gpu_main(args):
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded generator; no dataset or trained weights)",
         "config": {**workload_desc(wl), "parallelism": f"replicas x{world} (no exchange step)",
+                   "inputs_sha256": input_hashes(g.host),
                    **({"l2": f"{getattr(g, 'rotating_copies', 0)} rotating copies of the requantised weight "
                              f"(>= 3x L2) across the K steps of one CUDA-graph replay; e2e flushes L2 per step"}
                       if decode else {})},

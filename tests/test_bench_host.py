@@ -63,6 +63,13 @@ def test_reference_arm_json_line():
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "GB/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["e2e"]["h2d_bytes_per_step"] == 0
+    # every input buffer's SHA-256, reproducible from the seeded generator
+    from block_scaled_precision_requant_b200 import synth
+
+    hashes = line["config"]["inputs_sha256"]
+    assert hashes == bench.input_hashes(synth.make_workload("decode"))
+    assert sorted(hashes) == ["a_bf16", "scale2", "w_e4m3", "w_packed"]
+    assert all(len(v) == 64 and int(v, 16) >= 0 for v in hashes.values())
 
 
 def test_reference_arm_non_zero_rank_exits_quietly():
