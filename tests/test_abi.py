@@ -30,6 +30,35 @@ def test_header_declares_what_binding_wraps():
     assert _declared() == sorted(name for name, _, _ in bsr.SIGNATURES)
 
 
+def _header_defines():
+    src = open(HEADER).read()
+    out = {}
+    for name, val in re.findall(r"^#define (BSR_[A-Z0-9_]+) (.+)$", src, flags=re.M):
+        val = re.sub(r"(?<=\d)(u|LL|ULL)\b", "", val.split("/*")[0].strip())
+        if re.fullmatch(r"\d+", val):
+            out[name] = int(val)
+        elif m := re.fullmatch(r"\((\d+) << (\d+)\)", val):
+            out[name] = int(m.group(1)) << int(m.group(2))
+    return out
+
+
+def test_header_constants_match_the_binding(L):
+    # the binding restates a few header constants; they must agree (the
+    # reference's one test checks the same for its kernel constants)
+    d = _header_defines()
+    assert d["BSR_ABI_VERSION"] == bsr.abi_version()
+    assert d["BSR_DECODE_MAX_M"] == bsr.DECODE_MAX_M
+    assert d["BSR_DECODE_STATIC_WEIGHT"] == bsr.DECODE_STATIC_WEIGHT
+    assert d["BSR_MAX_SEGMENTS"] == bsr.MAX_SEGMENTS
+    assert d["BSR_MAX_DIM"] == 2 ** 31 - 1
+    assert d["BSR_NOALLOC_SCRATCH_BYTES"] == 16 << 20
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    enum = dict((int(v), "BSR_" + k) for k, v in re.findall(r"\bBSR_([A-Z]+) = (\d+)", src))
+    assert enum == bsr.STATUS_NAMES
+    common = open(os.path.join(ROOT, "block_scaled_precision_requant_b200", "csrc", "common.cuh")).read()
+    assert int(re.search(r"DEV_ERR_TIMEOUT_DEBUG = (\d+)", common).group(1)) == bsr.DEV_STATUS_DEBUG_WAIT
+
+
 def test_every_declared_symbol_is_exported(L):
     for name in _declared():
         assert hasattr(L, name), name
