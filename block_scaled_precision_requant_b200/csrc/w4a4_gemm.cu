@@ -95,10 +95,11 @@ constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl)
 
 // Shared-memory descriptor of a K-major, unswizzled source: 16-byte rows,
 // 8-row core matrices 128 bytes apart (the tcgen05.cp source of one atom).
+// The fields are those CuTe derives for this copy (LBO 16 B, SBO 128 B).
 __device__ __forceinline__ uint64_t smem_desc_k_plain(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
-  d |= (uint64_t)0 << 16;                     // leading byte offset: one core matrix along K
+  d |= (uint64_t)(16u >> 4) << 16;            // leading byte offset (one core matrix along K)
   d |= (uint64_t)(128u >> 4) << 32;           // stride byte offset: 8 rows x 16 B
   d |= (uint64_t)1 << 46;                     // descriptor version (sm_100)
   return d;                                   // layout type 0: no swizzle
