@@ -41,6 +41,7 @@
 
 #include "bsr.h"
 #include "common.cuh"
+#include "w4a4_desc.cuh"
 
 namespace bsr {
 // Records the message bsr_last_error() returns on this thread (api.cu).
@@ -70,15 +71,6 @@ constexpr uint32_t COL_SFA = ACC_BUFS * BN;        // 256
 constexpr uint32_t COL_SFB = COL_SFA + 4 * MMAS;   // 272
 static_assert(COL_SFB + 4 * MMAS <= TMEM_COLS, "tensor-memory plan");
 
-// Instruction descriptor of the block-scaled FP4 MMA: A and B E2M1 (format 1
-// of the FP4 kind), UE4M3 scales, both K-major, dense K = 64, scale ids 0.
-constexpr uint32_t idesc_mxf4(int m, int n) {
-  return (1u << 7)                        // A format: E2M1
-         | (1u << 10)                     // B format: E2M1
-         | ((uint32_t)(n >> 3) << 17)     // N / 8
-         | (0u << 23)                     // scale format: UE4M3
-         | ((uint32_t)(m >> 4) << 24);    // M / 16
-}
 constexpr uint32_t kIdesc = idesc_mxf4(BM, BN);
 
 struct Ctrl {
@@ -92,18 +84,6 @@ struct Ctrl {
 };
 
 constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(Ctrl);
-
-// Shared-memory descriptor of a K-major, unswizzled source: 16-byte rows,
-// 8-row core matrices 128 bytes apart (the tcgen05.cp source of one atom).
-// The fields are those CuTe derives for this copy (LBO 16 B, SBO 128 B).
-__device__ __forceinline__ uint64_t smem_desc_k_plain(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
-  d |= (uint64_t)(16u >> 4) << 16;            // leading byte offset (one core matrix along K)
-  d |= (uint64_t)(128u >> 4) << 32;           // stride byte offset: 8 rows x 16 B
-  d |= (uint64_t)1 << 46;                     // descriptor version (sm_100)
-  return d;                                   // layout type 0: no swizzle
-}
 
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
