@@ -669,7 +669,7 @@ def stacked_decode_extra(device, steps, peaks, cpu=True):
     return res
 
 
-def w4a16_extra(g, steps, cpu=True):
+def w4a16_extra(g, steps, peaks, cpu=True):
     """The NVFP4 W4A16 decode GEMV on the decode workload's weight as stored
     (0.5625 B per weight element): a CUDA-graph loop over rotating copies
     (>= 3x L2), bytes = N*K*0.5625 + 2MK + 2MN per step."""
@@ -699,6 +699,7 @@ def w4a16_extra(g, steps, cpu=True):
     del gr, ws
     g.check_status()
     res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
+           "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
            "note": "reads the NVFP4 weight as stored; not bit-compatible with the int8 path"}
     if cpu:
         import oracle
@@ -722,7 +723,7 @@ def oracle_seconds(fn, budget_s, max_calls=50):
     return spent / done, done
 
 
-def w4a4_extra(device, wl, host, steps, cpu=True):
+def w4a4_extra(device, wl, host, steps, peaks, cpu=True):
     """The NVFP4 W4A4 decode GEMV (activation rows quantised to NVFP4 inside
     the kernel) on the decode workload's weight as stored: a CUDA-graph loop
     over rotating copies (>= 3x L2), bytes = N*K*0.5625 + 2MK + 2MN per step."""
@@ -759,6 +760,7 @@ def w4a4_extra(device, wl, host, steps, cpu=True):
     if bsr.device_status() != 0:
         raise RuntimeError(f"device status word {bsr.device_status()}")
     res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
+           "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
            "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
     if cpu:
         import oracle
@@ -894,7 +896,7 @@ def gpu_main(args):
         kernel = "gemm_kernel"
     t_rw = g.timed_requant_w_only(min(args.steps, 20), args.warmup)
     g.check_status()
-    w4 = (w4a16_extra(g, max(args.steps, 20), cpu=not args.no_cpu)
+    w4 = (w4a16_extra(g, max(args.steps, 20), peaks, cpu=not args.no_cpu)
           if decode and not args.no_extra and world == 1 else None)
 
     ms_step, ms_e2e, ms_kernel, ms_rw, ms_e2e_eager = dist_max(
@@ -955,7 +957,7 @@ def gpu_main(args):
         if decode:
             line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks, cpu=not args.no_cpu)
             try:  # the last GPU work of the run: an error here costs only this entry
-                line["w4a4_decode"] = w4a4_extra(dev, wl, host, max(args.steps, 20), cpu=not args.no_cpu)
+                line["w4a4_decode"] = w4a4_extra(dev, wl, host, max(args.steps, 20), peaks, cpu=not args.no_cpu)
             except Exception as exc:  # noqa: BLE001 - reported in the line
                 line["w4a4_decode"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
     if rank == 0 and world == 1 and not args.no_cpu:
