@@ -1,6 +1,7 @@
 """GPU parity of the projection against the oracle.
 
-* block partials from the tensor cores: bit-exact,
+* block partials from the tensor cores: bit-exact (small ragged shapes, and
+  the M-tail tile of the 4095 x 8192 x 8192 workload at full K),
 * BF16 outputs of both paths (decode kernel, tcgen05 GEMM): within
   |err| <= 2^-7 |ref| + 1e-3 rms(ref),
 * the invariants: row bits independent of M and of the other rows (within a
@@ -54,6 +55,29 @@ def test_gemm_partials_bit_exact(shape):
     assert_close_bf16(bf16_bits(out), ref, "gemm output")
     # the dump variant and the plain kernel give the same output bits
     assert np.array_equal(bf16_bits(bsr.gemm(a_i8, a_st, w_i8, w_s)), bf16_bits(out))
+
+
+def test_gemm_partials_square_ragged_tail_tile():
+    # one 127 x 256 tile of the 4095 x 8192 x 8192 workload at full K: the
+    # last 127 activation rows (the ragged M tail, 4095 = 31 * 128 + 127) and
+    # the 256 weight rows around one of its x100 outlier rows.  Partials are
+    # per (m, n, block) and both requantisations are row-local, so this
+    # sub-problem is that tile of the full launch.
+    d = synth.make_workload("square_ragged")
+    m, n, k = d["workload"].shape
+    n0 = int(d["outlier_rows"][0]) // 256 * 256
+    w = {"w_packed": d["w_packed"][n0:n0 + 256], "w_e4m3": d["w_e4m3"][n0:n0 + 256], "scale2": d["scale2"]}
+    a = d["a_bits"][m - m % 128:]
+    assert a.shape == (127, k)
+    w_i8, w_s = _weights(w)
+    a_i8, a_st = bsr.requant_a(up_bf16(a))
+    out, p = bsr.gemm_partials(a_i8, a_st, w_i8, w_s)
+    qa, sa = oracle.requant_a(a)
+    qw, sw = _oracle_w(w, k)
+    ref_p = oracle.block_partials(qa, qw)
+    assert np.array_equal(p.cpu().numpy().astype(np.int64), ref_p)
+    assert_close_bf16(bf16_bits(out), oracle.bf16_rne(oracle.accumulate(ref_p, sa, sw)), "tail tile output")
+    assert bsr.device_status() == 0
 
 
 # --------------------------------------------------------------------------- both paths
