@@ -112,6 +112,30 @@ def test_whole_oracle_vs_float64_gemm_random(shape, recipe):
     _check_against_f64(a, w)
 
 
+@pytest.mark.parametrize("name", ["decode", "ffn_up", "ffn_down", "square_ragged"])
+def test_whole_oracle_vs_float64_gemm_workloads(name):
+    # the decode workload (1 x 4096 x 4096) in full; the prefill workloads on
+    # sampled outputs: sampled activation rows (ends, the ragged tail, the
+    # zero row or a row with near-zero groups) against three 128-row weight
+    # windows (first, last, and around an outlier row when there is one).
+    # Both requantisations are row-local, so each sampled output is computed
+    # exactly as in the full problem.
+    d = synth.make_workload(name)
+    m, n, k = d["workload"].shape
+    if name == "decode":
+        _check_against_f64(d["a_bits"], d)
+        return
+    info = d["act_info"]
+    must = [info["zero_row"]] if "zero_row" in info else []
+    if "near_zero_groups" in info:
+        must.append(int(info["near_zero_groups"][0]) // (k // 32))
+    rows = synth.sample_rows(m, 4, d["workload"].seed, must=must)
+    starts = [0, n - 128] + ([int(d["outlier_rows"][0]) // 128 * 128] if len(d["outlier_rows"]) else [])
+    for n0 in starts:
+        w = {"w_packed": d["w_packed"][n0:n0 + 128], "w_e4m3": d["w_e4m3"][n0:n0 + 128], "scale2": d["scale2"]}
+        _check_against_f64(d["a_bits"][rows], w)
+
+
 def test_row_bits_independent_of_m_and_other_rows(tiny):
     k = tiny["a_bits"].shape[1]
     w_i8, w_scale = oracle.requant_w(tiny["w_packed"], tiny["w_e4m3"], tiny["scale2"], k)
