@@ -1,7 +1,8 @@
 """GPU parity of the projection against the oracle.
 
-* block partials from the tensor cores: bit-exact (small ragged shapes, and
-  the M-tail tile of the 4095 x 8192 x 8192 workload at full K),
+* block partials from the tensor cores: bit-exact (small ragged shapes, the
+  16 x 256 x 512 workload in full, and the M-tail tile of the
+  4095 x 8192 x 8192 workload at full K),
 * BF16 outputs of both paths (decode kernel, tcgen05 GEMM): within
   |err| <= 2^-7 |ref| + 1e-3 rms(ref),
 * the invariants: row bits independent of M and of the other rows (within a
@@ -55,6 +56,19 @@ def test_gemm_partials_bit_exact(shape):
     assert_close_bf16(bf16_bits(out), ref, "gemm output")
     # the dump variant and the plain kernel give the same output bits
     assert np.array_equal(bf16_bits(bsr.gemm(a_i8, a_st, w_i8, w_s)), bf16_bits(out))
+
+
+def test_gemm_partials_tiny_workload_in_full(tiny):
+    # the 16 x 256 x 512 workload's own inputs, every partial
+    k = 512
+    w_i8, w_s = _weights(tiny)
+    a_i8, a_st = bsr.requant_a(up_bf16(tiny["a_bits"]))
+    out, p = bsr.gemm_partials(a_i8, a_st, w_i8, w_s)
+    qa, sa = oracle.requant_a(tiny["a_bits"])
+    qw, sw = _oracle_w(tiny, k)
+    ref_p = oracle.block_partials(qa, qw)
+    assert np.array_equal(p.cpu().numpy().astype(np.int64), ref_p)
+    assert_close_bf16(bf16_bits(out), oracle.bf16_rne(oracle.accumulate(ref_p, sa, sw)), "tiny workload")
 
 
 def test_gemm_partials_square_ragged_tail_tile():
