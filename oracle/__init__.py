@@ -24,7 +24,8 @@ Sources (the launcher pages of the ``metrale_model_layers`` ops crate):
 * ``w8a8_decode/parts.rs`` -- doc comment of ``W8a8Weight::segment``: a
   segment of a stacked weight yields the bits the stacked launch yields for
   those rows; ``W8a8Kernels::quant_silu``: the SiLU.mul quantiser (its
-  arithmetic is this module's reading, see ``silu_mul_bf16``).
+  arithmetic is this module's reading, see ``silu_mul_bf16``: the exact
+  product rounded once to BF16, then requant_a).
 * ``gemv_sw.rs`` -- the ``w4a16_gemv`` / ``w4a16_gemv_sw`` launches: the NVFP4
   W4A16 decode GEMV's arguments (its arithmetic is this module's reading, see
   ``w4a16_gemv``).
@@ -69,7 +70,7 @@ __all__ = [
     "bf16_rne",
     "proj_rows",
     "proj",
-    "exp_f32",
+    "f64_to_bf16_bits",
     "silu_mul_bf16",
     "requant_silu_a",
     "w4a16_gemv",
@@ -262,61 +263,40 @@ def proj(a_bits, w_packed, w_e4m3, scale2, k: int) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 # float32 constants, by bit pattern
-_LOG2E = np.uint32(0x3FB8AA3B).view(np.float32)    # 1.442695
-_LN2_HI = np.uint32(0x3F317200).view(np.float32)   # 0.693145751953125 (15 significant bits)
-_LN2_LO = np.uint32(0x35BFBE8E).view(np.float32)   # ln 2 - _LN2_HI
-_EXP_COEF = [np.uint32(b).view(np.float32) for b in
-             (0x3F800000, 0x3F800000, 0x3F000000, 0x3E2AAAAB, 0x3D2AAAAB, 0x3C088889, 0x3AB60B61)]  # 1/i!
+def f64_to_bf16_bits(x) -> np.ndarray:
+    """BF16 bits of float64 values rounded once to nearest, ties to even.
 
-
-def _pow2_f32(h: np.ndarray) -> np.ndarray:
-    """2^h as float32 for integer h in [-126, 127] (exact)."""
-    return ((h.astype(np.int64) + 127) << 23).astype(np.uint32).view(np.float32)
-
-
-def exp_f32(x) -> np.ndarray:
-    """exp in float32 by Cody-Waite range reduction and a degree-6 Taylor
-    polynomial, every operation a float32 multiply or add rounded to nearest
-    (no fused multiply-add):
-
-        n = rint_half_even(x * log2e)
-        r = (x - n * ln2_hi) - n * ln2_lo          (n * ln2_hi is exact)
-        p = 1 + r(1 + r(1/2 + r(1/6 + r(1/24 + r(1/120 + r/720)))))   (Horner)
-        exp(x) = (p * 2^h1) * 2^h2,  h1 = floor(n/2), h2 = n - h1
-
-    x > 88 gives +inf, x < -88 gives +0, NaN stays NaN."""
-    x = np.asarray(x, dtype=np.float32)
-    f32 = np.float32
-    with np.errstate(over="ignore", invalid="ignore", under="ignore"):
-        xc = np.clip(x, f32(-88.0), f32(88.0))
-        xc = np.where(np.isnan(xc), f32(0.0), xc).astype(np.float32)
-        n = np.rint((xc * _LOG2E).astype(np.float32)).astype(np.float32)
-        r = ((xc - (n * _LN2_HI).astype(np.float32)).astype(np.float32) - (n * _LN2_LO).astype(np.float32))
-        r = r.astype(np.float32)
-        p = _EXP_COEF[6]
-        for c in _EXP_COEF[5::-1]:
-            p = ((p * r).astype(np.float32) + c).astype(np.float32)
-        ni = n.astype(np.int64)
-        h1 = ni >> 1
-        h2 = ni - h1
-        y = ((p * _pow2_f32(h1)).astype(np.float32) * _pow2_f32(h2)).astype(np.float32)
-    y = np.where(x > f32(88.0), f32(np.inf), y)
-    y = np.where(x < f32(-88.0), f32(0.0), y)
-    return np.where(np.isnan(x), x, y).astype(np.float32)
+    The value goes to float32 rounded to odd (round to nearest, then, when
+    that was inexact and landed on an even significand, step one float32 ulp
+    towards the value), then to BF16 by bf16_rne.  With 16 more significand
+    bits in float32 than in BF16, rounding to odd first makes the second
+    rounding equal to one direct rounding of the float64 value.  BF16 has
+    float32's exponent range, so subnormal results follow the same rule."""
+    x = np.asarray(x, dtype=np.float64)
+    with np.errstate(over="ignore", invalid="ignore"):
+        f = x.astype(np.float32)
+        inexact = np.isfinite(f) & (f.astype(np.float64) != x)
+        even = (f.view(np.uint32) & np.uint32(1)) == 0
+        fix = inexact & even
+        toward = np.where(x > f.astype(np.float64), np.float32(np.inf), np.float32(-np.inf)).astype(np.float32)
+        f = np.where(fix, np.nextafter(f, toward), f).astype(np.float32)
+    return bf16_rne(f)
 
 
 def silu_mul_bf16(g_bits: np.ndarray, u_bits: np.ndarray) -> np.ndarray:
-    """BF16 bits of silu(g) * u from BF16 g and u (bit patterns):
-    e = exp_f32(-g), s = g / (1 + e), x = s * u, each rounded to float32, then
-    bf16_rne(x)."""
-    g = bf16_bits_to_f32(np.asarray(g_bits, dtype=np.uint16))
-    u = bf16_bits_to_f32(np.asarray(u_bits, dtype=np.uint16))
+    """BF16 bits of silu(g) * u from BF16 g and u (bit patterns): the
+    mathematical function silu(g) = g / (1 + e^-g) times u, evaluated in
+    float64 and rounded once to BF16 (round to nearest, ties to even).
+
+    float64 carries 29 bits more than float32, so the only values this can
+    misround are those within a few float64 ulps of a BF16 rounding boundary.
+    For g < -709.78 e^-g overflows float64 and the quotient is -0; the exact
+    product there is below 10^-300 * |u|, which rounds to zero in BF16."""
+    g = bf16_bits_to_f32(np.asarray(g_bits, dtype=np.uint16)).astype(np.float64)
+    u = bf16_bits_to_f32(np.asarray(u_bits, dtype=np.uint16)).astype(np.float64)
     with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
-        e = exp_f32(-g)
-        d = (np.float32(1.0) + e).astype(np.float32)
-        s = (g / d).astype(np.float32)
-        x = (s * u).astype(np.float32)
-    return bf16_rne(x)
+        x = g / (1.0 + np.exp(-g)) * u
+    return f64_to_bf16_bits(x)
 
 
 def requant_silu_a(g_bits: np.ndarray, u_bits: np.ndarray):

@@ -1,17 +1,23 @@
-"""Pins of the oracle's SiLU.mul quantiser (oracle.exp_f32, silu_mul_bf16,
-requant_silu_a) against mathematics, not against itself:
+"""Pins of the oracle's SiLU.mul quantiser (oracle.f64_to_bf16_bits,
+silu_mul_bf16, requant_silu_a) against mathematics, not against itself:
 
-* exp_f32 against float64 exp: within 3 float32 ulps over [-88, 88]
-  (measured worst 2.95), exact at 0, monotone, and the stated behaviour
-  outside the range;
-* silu(g) * u against a float64 evaluation of g / (1 + e^-g) * u rounded once
-  to BF16: equal except at BF16 rounding boundaries, where they may differ by
-  one BF16 step;
-* closed forms: silu(0) = 0, silu(g) = g for large g, silu(g) = -0 for very
-  negative g;
-* the quantiser: requant_a of the float64 product's BF16 gives the same codes
-  and scales.
+* f64_to_bf16_bits against a direct search of the table of every finite
+  BF16 value (nearest, ties to the even bit pattern), on random values, on
+  exact BF16 midpoints and on values one float64 ulp either side of them --
+  the cases a plain float64 -> float32 -> BF16 double rounding gets wrong;
+* silu(g) * u against a 50-digit decimal evaluation of g / (1 + e^-g) * u,
+  rounded to BF16 with exact rational comparisons: equal bits everywhere
+  (the float64 evaluation is accurate to a few float64 ulps, and no sampled
+  value lies that close to a BF16 rounding boundary -- the test checks that
+  too);
+* closed forms: silu(0) = 0, silu(g) * u = g * u for large g, and a very
+  negative g gives a signed zero;
+* the quantiser: requant_a of the decimal reference's BF16 product gives the
+  same codes and scales.
 """
+from decimal import Decimal, getcontext
+from fractions import Fraction
+
 import numpy as np
 
 import oracle
@@ -27,77 +33,119 @@ def _val(bits):
     return oracle.bf16_bits_to_f32(bits).astype(np.float64)
 
 
-def test_exp_within_three_ulp_of_float64():
-    x = np.linspace(-88.0, 88.0, 400_001).astype(np.float32)
-    got = oracle.exp_f32(x).astype(np.float64)
-    ref = np.exp(x.astype(np.float64))
-    ulp = np.maximum(np.spacing(np.abs(ref.astype(np.float32))).astype(np.float64), 2.0 ** -149)
-    err = np.abs(got - ref) / ulp
-    assert err.max() <= 3.0, (float(err.max()), float(x[np.argmax(err)]))
-    assert np.all(np.diff(got) >= 0), "exp_f32 must be monotone"
+# Every finite non-negative BF16 value, ascending, with its bit pattern.
+_POS_BITS = np.arange(0x0000, 0x7F80, dtype=np.uint16)
+_POS_VALS = _val(_POS_BITS)
 
 
-def test_exp_special_values():
-    x = np.array([0.0, 88.0, 88.5, 1e30, -88.0, -88.5, -1e30, np.inf, -np.inf, np.nan], dtype=np.float32)
-    y = oracle.exp_f32(x)
-    assert y[0] == F32(1.0)
-    assert np.isfinite(y[1]) and y[1] > F32(1e38)
-    assert np.isinf(y[2]) and np.isinf(y[3]) and np.isinf(y[7])
-    assert 0.0 < y[4] < 1e-37  # exp(-88) is subnormal in float32
-    assert y[5] == 0.0 and y[6] == 0.0 and y[8] == 0.0
-    assert np.isnan(y[9])
+def _nearest_bf16_exact(x: Fraction) -> int:
+    """BF16 bits nearest to the rational x (ties to the even pattern),
+    by search in the value table; beyond the largest finite value halfway
+    to 2^128, infinity."""
+    sign = 0x8000 if x < 0 else 0
+    a = -x if x < 0 else x
+    top = Fraction(_POS_VALS[-1]) + (Fraction(2) ** 128 - Fraction(_POS_VALS[-1])) / 2
+    if a > top or (a == top and (int(_POS_BITS[-1]) & 1)):
+        return sign | 0x7F80
+    i = int(np.searchsorted(_POS_VALS, float(a), side="right")) - 1
+    i = max(0, min(i, len(_POS_VALS) - 1))
+    # float(a) may round across a table entry; settle with exact comparisons
+    while i + 1 < len(_POS_VALS) and Fraction(_POS_VALS[i + 1]) <= a:
+        i += 1
+    while i > 0 and Fraction(_POS_VALS[i]) > a:
+        i -= 1
+    lo = Fraction(_POS_VALS[i])
+    if lo == a or i + 1 == len(_POS_VALS):
+        return sign | int(_POS_BITS[i])
+    hi = Fraction(_POS_VALS[i + 1])
+    d_lo, d_hi = a - lo, hi - a
+    if d_lo < d_hi or (d_lo == d_hi and (int(_POS_BITS[i]) & 1) == 0):
+        return sign | int(_POS_BITS[i])
+    return sign | int(_POS_BITS[i + 1])
 
 
-def _reference_product_bits(g_bits, u_bits):
+def test_f64_to_bf16_random_values():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(3000) * 10.0 ** rng.uniform(-40, 38, 3000)
+    got = oracle.f64_to_bf16_bits(x)
+    want = np.array([_nearest_bf16_exact(Fraction(float(v))) for v in x], dtype=np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_f64_to_bf16_midpoints_and_neighbours():
+    rng = np.random.default_rng(2)
+    bits = rng.integers(0x0001, 0x7F7F, size=400).astype(np.uint16)
+    lo = _val(bits)
+    hi = _val(bits + 1)
+    mid = (lo + hi) / 2  # exact in float64
+    vals = np.concatenate([mid, np.nextafter(mid, np.inf), np.nextafter(mid, -np.inf)])
+    vals = np.concatenate([vals, -vals])
+    got = oracle.f64_to_bf16_bits(vals)
+    want = np.array([_nearest_bf16_exact(Fraction(float(v))) for v in vals], dtype=np.uint16)
+    assert np.array_equal(got, want)
+    # the double rounding this guards against does differ on some of them
+    naive = oracle.bf16_rne(vals.astype(np.float32))
+    assert np.any(naive != want)
+
+
+def _silu_mul_decimal(g: float, u: float) -> Fraction:
+    getcontext().prec = 50
+    dg = Decimal(g)
+    val = dg / (Decimal(1) + (-dg).exp()) * Decimal(u)
+    return Fraction(val)
+
+
+def _reference_bits(g_bits, u_bits):
     g = _val(g_bits)
     u = _val(u_bits)
-    with np.errstate(over="ignore"):
-        ref = g / (1.0 + np.exp(-g)) * u  # float64
-    return _bf16(ref.astype(np.float32))  # float64 -> float32 -> bf16
+    return np.array([_nearest_bf16_exact(_silu_mul_decimal(float(a), float(b))) for a, b in zip(g, u)],
+                    dtype=np.uint16)
 
 
-def _assert_product_close(got, want):
-    same = got == want
-    if not np.all(same):
-        # only BF16 rounding boundaries may differ, by one BF16 step
-        a = got[~same].astype(np.int32)
-        b = want[~same].astype(np.int32)
-        assert np.all(np.abs(a - b) == 1), "product differs by more than one BF16 step"
-        assert (~same).mean() < 1e-3, f"{int((~same).sum())} of {same.size} products differ"
+def _distance_to_boundary(x: Fraction) -> Fraction:
+    """Relative distance from x to the nearest BF16 rounding boundary."""
+    if x == 0:
+        return Fraction(1)
+    b = _nearest_bf16_exact(x)
+    v = Fraction(float(_val(np.array([b], dtype=np.uint16))[0]))
+    step = Fraction(float(_val(np.array([(b & 0x7FFF) + 1], dtype=np.uint16))[0])) - abs(v)
+    return abs(step / 2 - abs(x - v)) / abs(x)
 
 
-def test_silu_of_grid_matches_float64():
-    g_bits = _bf16(np.linspace(-30.0, 30.0, 200_001))
-    u_bits = _bf16(np.ones(g_bits.shape))
-    _assert_product_close(oracle.silu_mul_bf16(g_bits, u_bits), _reference_product_bits(g_bits, u_bits))
-
-
-def test_silu_mul_random_matches_float64():
+def test_silu_mul_matches_decimal_reference():
     rng = np.random.default_rng(7)
-    g_bits = _bf16(rng.standard_normal(200_000) * 3)
-    u_bits = _bf16(rng.standard_normal(200_000) * 2)
-    _assert_product_close(oracle.silu_mul_bf16(g_bits, u_bits), _reference_product_bits(g_bits, u_bits))
+    g_bits = _bf16(np.concatenate([rng.standard_normal(1500) * 3, np.linspace(-120.0, 120.0, 500)]))
+    u_bits = _bf16(rng.standard_normal(2000) * 10.0 ** rng.uniform(-3, 3, 2000))
+    got = oracle.silu_mul_bf16(g_bits, u_bits)
+    want = _reference_bits(g_bits, u_bits)
+    # no sampled product lies within 2^-40 (relative) of a rounding boundary,
+    # so the float64 evaluation must round the same way
+    gs, us = _val(g_bits), _val(u_bits)
+    for a, b in zip(gs[:200], us[:200]):
+        assert _distance_to_boundary(_silu_mul_decimal(float(a), float(b))) > Fraction(1, 2 ** 40)
+    assert np.array_equal(got, want)
 
 
 def test_silu_closed_forms():
     u = _bf16(np.array([1.5, -2.0, 3.0, 0.75], dtype=np.float32))
     x = _val(oracle.silu_mul_bf16(_bf16(np.zeros(4)), u))
     assert np.all(x == 0.0)
-    g = _bf16(np.full(4, 40.0))  # 1 + e^-40 rounds to 1 in float32
+    g = _bf16(np.full(4, 40.0))  # e^-40 < 2^-57: silu(40) = 40 (1 - 4e-18)
     assert np.array_equal(oracle.silu_mul_bf16(g, u), _bf16(_val(g) * _val(u)))
-    g = _bf16(np.full(4, -100.0))  # e^100 overflows: g / inf = -0
-    x = _val(oracle.silu_mul_bf16(g, u))
-    assert np.all(x == 0.0)
+    g = _bf16(np.full(4, -100.0))  # |silu(-100)| = 3.7e-42, far below half the smallest BF16 subnormal
+    got = oracle.silu_mul_bf16(g, u)
+    assert np.array_equal(got, np.array([0x8000, 0x0000, 0x8000, 0x8000], dtype=np.uint16))
+    g = _bf16(np.full(4, -89.0))  # silu(-89) = -89 e^-89 = -3.9e-37: a normal BF16 value, not zero
+    assert np.all(_val(oracle.silu_mul_bf16(g, u)) != 0.0)
 
 
-def test_quantiser_is_requant_of_the_product():
+def test_quantiser_is_requant_of_the_exact_product():
     rng = np.random.default_rng(11)
     m, k = 5, 96
     g_bits = _bf16(rng.standard_normal((m, k)) * 2)
     u_bits = _bf16(rng.standard_normal((m, k)))
     q, s = oracle.requant_silu_a(g_bits, u_bits)
-    ref_bits = _reference_product_bits(g_bits, u_bits)
-    assert np.array_equal(oracle.silu_mul_bf16(g_bits, u_bits), ref_bits)  # no rounding boundary hit here
+    ref_bits = _reference_bits(g_bits.reshape(-1), u_bits.reshape(-1)).reshape(m, k)
     q2, s2 = oracle.requant_a(ref_bits)
     assert np.array_equal(q, q2) and np.array_equal(s.view(np.uint32), s2.view(np.uint32))
     assert q.dtype == np.int8 and q.shape == (m, k) and s.shape == (m, k // 32)
