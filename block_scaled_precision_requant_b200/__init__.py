@@ -55,6 +55,9 @@ __all__ = [
     "sf_blocked_bytes",
     "sf_blocked",
     "w4a4_gemm",
+    "w4a4_proj",
+    "gemm_block_m",
+    "w4a4_proj_scratch_bytes",
     "silu_mul",
     "requant_silu_a",
     "proj_silu_scratch_bytes",
@@ -91,6 +94,7 @@ SIGNATURES = [
     ("bsr_requant_a", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_gemm", ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_proj_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
+    ("bsr_gemm_block_m", ctypes.c_int, [_I64, _I64]),
     ("bsr_proj", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_decode", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_gemm_partials", ctypes.c_int, [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _P]),
@@ -105,6 +109,8 @@ SIGNATURES = [
     ("bsr_nvfp4_sf_blocked_bytes", ctypes.c_size_t, [_I64, _I64]),
     ("bsr_nvfp4_sf_blocked", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     ("bsr_w4a4_gemm", ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P, _P]),
+    ("bsr_w4a4_proj_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
+    ("bsr_w4a4_proj", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_silu_mul", ctypes.c_int, [_P, _P, _P, _I64, _I64, _P]),
     ("bsr_requant_silu_a", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_proj_silu_scratch_bytes", ctypes.c_size_t, [_I64, _I64]),
@@ -630,3 +636,44 @@ def w4a4_gemm(a_packed, a_sf_blocked, a_scale2, w_packed, w_sf_blocked, scale2: 
         )
     )
     return out
+
+
+def w4a4_proj_scratch_bytes(m: int, k: int) -> int:
+    """Scratch bytes of :func:`w4a4_proj` for M rows (0 if invalid)."""
+    return int(lib().bsr_w4a4_proj_scratch_bytes(m, k))
+
+
+def w4a4_proj(a, w_packed, w_sf_blocked, scale2: float, out=None, scratch=None, stream=None):
+    """The W4A4 projection on the tensor cores: a [M, K] bfloat16 quantised to
+    NVFP4 rows, scales relaid, FP4 MMA against w_packed [N, K/2] (scales
+    w_sf_blocked from :func:`sf_blocked`) -> out [M, N] bfloat16."""
+    torch = _torch()
+    m, k = a.shape
+    n = w_packed.shape[0]
+    if out is None:
+        out = _empty((m, n), torch.bfloat16, a)
+    need = w4a4_proj_scratch_bytes(m, k)
+    if scratch is None:
+        scratch = _empty((max(need, 1),), torch.uint8, a)
+    _check(
+        lib().bsr_w4a4_proj(
+            _dev(a, torch.bfloat16, (m, k), "a"),
+            _dev(w_packed, torch.uint8, (n, k // 2), "w_packed"),
+            _dev(w_sf_blocked, torch.uint8, (sf_blocked_bytes(n, k),), "w_sf_blocked"),
+            ctypes.c_float(float(scale2)),
+            _dev(out, torch.bfloat16, (m, n), "out"),
+            m,
+            n,
+            k,
+            ctypes.c_void_p(scratch.data_ptr()),
+            scratch.numel() * scratch.element_size(),
+            _stream_ptr(stream),
+        )
+    )
+    return out
+
+
+def gemm_block_m(m: int, n: int) -> int:
+    """Activation rows per tile the tensor-core GEMM uses for M x N on the
+    current device (128, 192 or 256; 0 without a usable device)."""
+    return int(lib().bsr_gemm_block_m(m, n))

@@ -123,36 +123,67 @@ int64_t a_scale_ld(int64_t m) { return (m + 3) / 4 * 4; }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
-                     uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream,
+// Everything one GEMM launch needs, prepared -- and every check that can
+// fail done -- before anything is queued.
+struct GemmPlan {
+  bsr::GemmMaps maps;
+  DevInfo d;
+  int m = 0, n = 0, k = 0, bm = 0;
+  long long ldo = 0;
+  int max_ctas = 0;
+};
+
+bsr_status gemm_plan(GemmPlan& p, const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8,
+                     const float* w_scale, uint16_t* out, bool partials, int64_t m, int64_t n, int64_t k,
                      int64_t ldo = -1, int max_ctas = 0) {
   if (ldo < 0) ldo = n;
   bsr_status st = check_dims(m, n, k, true, true);
   if (st != BSR_OK) return st;
   if (k % 128 != 0) return fail(BSR_ESHAPE, "bsr_gemm needs K %% 128 == 0 (K=%lld)", (long long)k);
-  if (m == 0 || n == 0) return ok();
   if (!a_i8 || !a_scale_t || !w_i8 || !w_scale || !out) return fail(BSR_EINVAL, "null pointer");
   if (!aligned16(a_i8) || !aligned16(a_scale_t) || !aligned16(w_i8) || !aligned16(w_scale) ||
       (reinterpret_cast<uintptr_t>(out) & 1u))
     return fail(BSR_EALIGN, "bsr_gemm: pointers must be 16-byte aligned (out: 2-byte)");
-  DevInfo d;
-  if ((st = device_info(d)) != BSR_OK) return st;
-  if (bsr::gemm_smem_bytes() > d.smem_optin)
-    return fail(BSR_ENODEV, "device shared memory %zu < %zu", d.smem_optin, bsr::gemm_smem_bytes());
-  bsr::GemmMaps maps;
+  if ((st = device_info(p.d)) != BSR_OK) return st;
+  if (bsr::gemm_smem_bytes() > p.d.smem_optin)
+    return fail(BSR_ENODEV, "device shared memory %zu < %zu", p.d.smem_optin, bsr::gemm_smem_bytes());
+  const uint32_t bm = (uint32_t)bsr::gemm_block_m(m, n, p.d.num_sms);
+  cudaError_t e = bsr::gemm_prepare_device(partials, (int)bm);
+  if (e != cudaSuccess) return fail(BSR_ECUDA, "gemm shared-memory opt-in: %s", cudaGetErrorString(e));
   const int64_t nb = k / 32;
-  if ((st = encode_2d(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_i8, k, n, k, 128, 128,
+  if ((st = encode_2d(&p.maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, w_i8, k, n, k, bsr::kGemmBoxK, bsr::kGemmBoxW,
                       CU_TENSOR_MAP_SWIZZLE_128B, "w_i8")) != BSR_OK ||
-      (st = encode_2d(&maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_i8, k, m, k, 128, 128,
+      (st = encode_2d(&p.maps.a, CU_TENSOR_MAP_DATA_TYPE_UINT8, a_i8, k, m, k, bsr::kGemmBoxK, bm,
                       CU_TENSOR_MAP_SWIZZLE_128B, "a_i8")) != BSR_OK ||
-      (st = encode_2d(&maps.ws, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w_scale, nb, n, nb * 4, 4, 128,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, "w_scale")) != BSR_OK ||
-      (st = encode_2d(&maps.as, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a_scale_t, m, nb, a_scale_ld(m) * 4, 128, 4,
-                      CU_TENSOR_MAP_SWIZZLE_NONE, "a_scale_t")) != BSR_OK)
+      (st = encode_2d(&p.maps.ws, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w_scale, nb, n, nb * 4, bsr::kGemmBoxKB,
+                      bsr::kGemmBoxW, CU_TENSOR_MAP_SWIZZLE_NONE, "w_scale")) != BSR_OK ||
+      (st = encode_2d(&p.maps.as, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a_scale_t, m, nb, a_scale_ld(m) * 4,
+                      bm, bsr::kGemmBoxKB, CU_TENSOR_MAP_SWIZZLE_NONE, "a_scale_t")) != BSR_OK)
     return st;
-  return cuda_status(bsr::launch_gemm(maps, out, partials, d.status, (int)m, (int)n, (int)k, (long long)ldo,
-                                      as_stream(stream), d.num_sms, max_ctas),
+  p.m = (int)m;
+  p.n = (int)n;
+  p.k = (int)k;
+  p.bm = (int)bm;
+  p.ldo = (long long)ldo;
+  p.max_ctas = max_ctas;
+  return BSR_OK;
+}
+
+bsr_status gemm_run(const GemmPlan& p, uint16_t* out, int32_t* partials, void* stream) {
+  return cuda_status(bsr::launch_gemm(p.maps, out, partials, p.d.status, p.m, p.n, p.k, p.bm, p.ldo,
+                                      as_stream(stream), p.d.num_sms, p.max_ctas),
                      "gemm launch");
+}
+
+bsr_status gemm_impl(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_i8, const float* w_scale,
+                     uint16_t* out, int32_t* partials, int64_t m, int64_t n, int64_t k, void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (k % 128 != 0) return fail(BSR_ESHAPE, "bsr_gemm needs K %% 128 == 0 (K=%lld)", (long long)k);
+  if (m == 0 || n == 0) return ok();
+  GemmPlan p;
+  if ((st = gemm_plan(p, a_i8, a_scale_t, w_i8, w_scale, out, partials != nullptr, m, n, k)) != BSR_OK) return st;
+  return gemm_run(p, out, partials, stream);
 }
 
 bsr_status decode_mr(int64_t m, int64_t k, DevInfo& d, int& mr) {
@@ -249,6 +280,16 @@ bsr_status check_proj_args(const uint16_t* a, const int8_t* w_i8, const float* w
 }  // namespace
 
 namespace bsr {
+// Device address of the library's status word on the current device (the
+// word bsr_device_status() reads and clears).
+bsr_status library_status_word(int** out) {
+  DevInfo d;
+  const bsr_status st = device_info(d);
+  if (st != BSR_OK) return st;
+  *out = d.status;
+  return BSR_OK;
+}
+
 bsr_status report(bsr_status st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -315,6 +356,13 @@ bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const i
   return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, partials, m, n, k, stream);
 }
 
+int bsr_gemm_block_m(int64_t m, int64_t n) {
+  if (m < 1 || n < 1 || m > BSR_MAX_DIM || n > BSR_MAX_DIM) return 0;
+  DevInfo d;
+  if (device_info(d) != BSR_OK) return 0;
+  return bsr::gemm_block_m(m, n, d.num_sms);
+}
+
 size_t bsr_proj_scratch_bytes(int64_t m, int64_t k) {
   if (m <= BSR_DECODE_MAX_M || k <= 0 || k % 128 != 0) return 0;
   return align256((size_t)m * (size_t)k) + (size_t)(k / 32) * (size_t)a_scale_ld(m) * 4;
@@ -361,8 +409,14 @@ bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale,
   if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
   int8_t* a_i8 = static_cast<int8_t*>(scratch);
   float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
-  if ((st = bsr_requant_a(a, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
-  return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
+  // plan the GEMM (tensor maps, shared-memory opt-in) before the first launch
+  GemmPlan p;
+  if ((st = gemm_plan(p, a_i8, a_scale_t, w_i8, w_scale, out, false, m, n, k)) != BSR_OK) return st;
+  if ((st = cuda_status(bsr::launch_requant_a(a, a_i8, a_scale_t, (int)m, (int)k, (int)a_scale_ld(m),
+                                              as_stream(stream), p.d.num_sms),
+                        "requant_a launch")) != BSR_OK)
+    return st;
+  return gemm_run(p, out, nullptr, stream);
 }
 
 bsr_status bsr_silu_mul(const uint16_t* gate, const uint16_t* up, uint16_t* x, int64_t m, int64_t k, void* stream) {
@@ -414,14 +468,25 @@ bsr_status bsr_proj_silu(const uint16_t* gate, const uint16_t* up, const int8_t*
   if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
   if (m <= BSR_DECODE_MAX_M || k % 128 != 0) {
     // decode route: the BF16 product into scratch, then the decode kernel
+    // (its shared-memory fit is checked before the first launch)
     uint16_t* x = static_cast<uint16_t*>(scratch);
-    if ((st = bsr_silu_mul(gate, up, x, m, k, stream)) != BSR_OK) return st;
+    DevInfo d;
+    int mr = 0;
+    if ((st = decode_mr(m, k, d, mr)) != BSR_OK) return st;
+    if ((st = cuda_status(bsr::launch_silu_mul(gate, up, x, (int)m, (int)k, as_stream(stream), d.num_sms),
+                          "silu_mul launch")) != BSR_OK)
+      return st;
     return decode_impl(x, w_i8, w_scale, out, m, n, k, stream);
   }
   int8_t* a_i8 = static_cast<int8_t*>(scratch);
   float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
-  if ((st = bsr_requant_silu_a(gate, up, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
-  return gemm_impl(a_i8, a_scale_t, w_i8, w_scale, out, nullptr, m, n, k, stream);
+  GemmPlan p;
+  if ((st = gemm_plan(p, a_i8, a_scale_t, w_i8, w_scale, out, false, m, n, k)) != BSR_OK) return st;
+  if ((st = cuda_status(bsr::launch_requant_silu_a(gate, up, a_i8, a_scale_t, (int)m, (int)k, (int)a_scale_ld(m),
+                                                   as_stream(stream), p.d.num_sms),
+                        "requant_silu_a launch")) != BSR_OK)
+    return st;
+  return gemm_run(p, out, nullptr, stream);
 }
 
 bsr_status bsr_decode_stacked(const uint16_t* a, const int8_t* const* w_i8, const float* const* w_scale,
@@ -460,12 +525,12 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
   if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0) return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
   int8_t* a_i8 = static_cast<int8_t*>(scratch);
   float* a_scale_t = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)m * (size_t)k));
-  if ((st = bsr_requant_a(a, a_i8, a_scale_t, m, k, stream)) != BSR_OK) return st;
   // One GEMM per segment into its column slice of out (row stride = all
   // rows).  The segments run concurrently, each on a side stream forked from
   // and joined back into the caller's stream, with persistent grids sized in
   // proportion to their tile counts so that together they fill the SMs once
-  // (a small segment alone would leave most SMs idle).
+  // (a small segment alone would leave most SMs idle).  Every segment's plan
+  // and the side streams are made before the first launch.
   DevInfo d;
   if ((st = device_info(d)) != BSR_OK) return st;
   int dev = 0;
@@ -473,27 +538,36 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
   long long tiles[BSR_MAX_SEGMENTS] = {}, total_tiles = 0;
   for (int s = 0; s < num_segs; ++s) {
     const int64_t ns = segs.off[s + 1] - segs.off[s];
-    tiles[s] = ((ns + 127) / 128) * ((m + 127) / 128);
+    tiles[s] = bsr::gemm_tiles(m, ns, d.num_sms);
     total_tiles += tiles[s];
+  }
+  GemmPlan plans[BSR_MAX_SEGMENTS];
+  for (int s = 0; s < num_segs; ++s) {
+    if (tiles[s] == 0) continue;
+    int ctas = (int)((long long)d.num_sms * tiles[s] / total_tiles);
+    ctas = ctas < 1 ? 1 : ctas;
+    const int64_t ns = segs.off[s + 1] - segs.off[s];
+    if ((st = gemm_plan(plans[s], a_i8, a_scale_t, w_i8[s], w_scale[s], out + segs.off[s], false, m, ns, k, n,
+                        ctas)) != BSR_OK)
+      return st;
   }
   std::lock_guard<std::mutex> lk(g_stacked_mu);
   StackedStreams* ss = nullptr;
   if ((st = stacked_streams(dev, ss)) != BSR_OK) return st;
   cudaStream_t cs = as_stream(stream);
+  if ((st = cuda_status(bsr::launch_requant_a(a, a_i8, a_scale_t, (int)m, (int)k, (int)a_scale_ld(m), cs,
+                                              d.num_sms),
+                        "requant_a launch")) != BSR_OK)
+    return st;
   if (cudaEventRecord(ss->fork, cs) != cudaSuccess) return fail(BSR_ECUDA, "stacked fork record failed");
   for (int s = 0; s < num_segs; ++s) {
     if (tiles[s] == 0) continue;
-    int ctas = (int)((long long)d.num_sms * tiles[s] / total_tiles);
-    ctas = ctas < 1 ? 1 : ctas;
     if (cudaStreamWaitEvent(ss->side[s], ss->fork, 0) != cudaSuccess) return fail(BSR_ECUDA, "stacked fork wait failed");
-    const int64_t ns = segs.off[s + 1] - segs.off[s];
-    if ((st = gemm_impl(a_i8, a_scale_t, w_i8[s], w_scale[s], out + segs.off[s], nullptr, m, ns, k, ss->side[s], n,
-                        ctas)) != BSR_OK)
-      return st;
+    if ((st = gemm_run(plans[s], out + segs.off[s], nullptr, ss->side[s])) != BSR_OK) return st;
     if (cudaEventRecord(ss->join[s], ss->side[s]) != cudaSuccess) return fail(BSR_ECUDA, "stacked join record failed");
     if (cudaStreamWaitEvent(cs, ss->join[s], 0) != cudaSuccess) return fail(BSR_ECUDA, "stacked join wait failed");
   }
-  return BSR_OK;
+  return ok();
 }
 
 bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,

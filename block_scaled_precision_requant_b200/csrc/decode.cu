@@ -21,6 +21,8 @@
 // weight is one [N, K] tensor or a table of stacked segments.
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "quant.cuh"
@@ -275,6 +277,8 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
 
 static bool decode_scale_bulk(int k) { return (k % 128) == 0; }
 
+static std::mutex g_decode_optin_mu;
+
 // Rows per CTA: the largest power of two <= 16 that covers M and fits the
 // shared-memory budget together with at least one weight-row slot.
 int decode_rows_per_cta(int m, int k, size_t smem_limit) {
@@ -299,16 +303,20 @@ static cudaError_t launch_decode_t(const uint16_t* a, const Src& src, int n, uin
   w = w < 1 ? 1 : (w > kMaxW ? kMaxW : w);
   while (w > 1 && decode_smem_layout(MR, k, w, sb).total > smem_limit) --w;
   const size_t smem = decode_smem_layout(MR, k, w, sb).total;
-  // dynamic shared-memory limit granted so far, per device (per <MR, Src>)
+  // dynamic shared-memory limit granted so far, per device (per <MR, Src>),
+  // raised under a lock shared by all variants
   static size_t granted[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (smem > granted[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    granted[dev] = smem;
+  {
+    std::lock_guard<std::mutex> lk(g_decode_optin_mu);
+    if (smem > granted[dev]) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      granted[dev] = smem;
+    }
   }
   const int gy = (m + MR - 1) / MR;
   long long gx = (n + w - 1) / w;

@@ -4,31 +4,44 @@
 //   out[m, n] = bf16( sum_b  P[m, n, b] * a_scale[m, b] * w_scale[n, b] ),
 //   P[m, n, b] = sum_{j<32} a_i8[m, 32b+j] * w_i8[n, 32b+j]   (exact int32)
 //
-// Tile: 128 weight rows (tensor-memory lanes, MMA M) x 128 activation rows
-// (tensor-memory columns, MMA N).  Each 32-wide K block is ONE
-// `tcgen05.mma.kind::i8` (128x128x32) into its own int32 tensor-memory
-// buffer, because the scales change every 32 elements; a four-deep ring of
-// such buffers lets the MMA of block b+1..b+3 run while the epilogue warps
-// rescale block b into float32 register accumulators.
+// Tile: 128 weight rows (tensor-memory lanes, MMA M) x BM activation rows
+// (tensor-memory columns, MMA N), BM in {128, 192, 256}: 128 when M <= 128,
+// else the width whose whole waves of tiles take the least estimated time.  Each
+// 32-wide K block is ONE `tcgen05.mma.kind::i8` (128 x BM x 32) into its own
+// int32 tensor-memory buffer, because the scales change every 32 elements;
+// a ring of 512 / BM such buffers lets the MMA of the next block run while
+// the epilogue warps rescale this one into float32 register accumulators.
 //
-// Warp roles (640 threads, one CTA per SM, persistent over tiles):
+// The rescale is two FP32 FMAs per element and block on the CUDA cores, so
+// the kernel is bound by the FP32 pipe, not by the tensor pipe.  What decides
+// how close it gets to that bound is the instruction overhead per block
+// (barrier waits, tensor-memory loads, scale loads) against the FMAs it
+// feeds: each epilogue thread owns 4 weight rows x BM/8 activation columns,
+// so one wait, one buffer release and one weight-scale load serve BM/2 FMA
+// pairs.
+//
+// Warp roles (384 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: per stage (4 K blocks = 128 bytes of K) the W
-//               and A tiles (128x128 bytes, 128-byte swizzle) and their
-//               scale tiles, into a 5-stage shared-memory ring.
-//   warps 1, 3  MMA issuers (one thread each; K blocks 0,2 and 1,3 of a
-//               stage); warp 1 also allocates the tensor memory.
+//               and A tiles (128-byte swizzle) and their scale tiles, into a
+//               multi-stage shared-memory ring.
+//   warp 1      MMA issuer (one thread); also owns the tensor memory.
 //   warp 2      scale preparation: pre-multiplies the staged activation
-//               scales by 2^49 and the weight scales by 2^100, or flags the
-//               stage when a scale falls outside the exponent window of the
-//               fast epilogue (the stage then keeps its scales as loaded).
-//   warps 4-19  epilogue: four warps per 32-lane quarter of tensor memory,
-//               32 activation columns each, read with 16x128b loads (4
-//               weight rows x 8 activation columns per thread).
+//               scales by 2^49 and the weight scales by 2^100 and rewrites
+//               both tiles into the epilogue's read order, or flags the stage
+//               when a scale falls outside the exponent window of the fast
+//               epilogue (the stage then keeps its scales as loaded).
+//   warp 3      idle.
+//   warps 4-11  epilogue: warp w reads tensor-memory lanes 32(w%4).. (the
+//               quarter it may access) and the half (w-4)/4 of the columns,
+//               in chunks of 16 columns with 16x128b loads, the next chunk's
+//               load in flight while the current one is rescaled: a thread
+//               holds weight rows 32q + t/4 + 8i (i = 0..3) x columns
+//               c + t%4 + 4k.
 //
 // Epilogue arithmetic (per element and block, exact up to one rounding in
 // each of two FMAs):
 //   Every K block is two MMAs into the same buffer: first a u8 x u8 MMA of
-//   two constant tiles of 128s with accumulation off (32*128*128 = 2^19),
+//   two constant operands of 128s with accumulation off (32*128*128 = 2^19),
 //   then the s8 x s8 MMA of the data with accumulation on, so the
 //   accumulator holds P' = P + 2^19, which lies in [8160, 1040416] because
 //   |P| <= 32*127*127 = 516128 < 2^19.  Read as a float32 bit pattern, P' is
@@ -41,9 +54,16 @@
 //   needs W in [2^23, 2^128) and a_scale * 2^49 finite, i.e. nonzero
 //   |w_scale| in [2^-77, 2^28) and a_scale < 2^79; a stage with any scale
 //   outside that window (or NaN) takes the plain path (convert, multiply,
-//   fma) for all its blocks.  Two FMAs per element run as packed f32x2 FMAs.
+//   fma) for all its blocks.  Registers (l, l+8) of a 16x128b load are two
+//   weight rows at one column: the operand pair of one packed f32x2 FMA.
+//
+// Failure handling: every wait is bounded.  A wait that runs out raises the
+// CTA's abort flag and a bit in the status word; the TMA thread then waits
+// (bounded) for the copies it issued, the MMA thread commits and waits for
+// its issued MMAs, and only then does the CTA free its tensor memory.
 #include <cuda_bf16.h>
 
+#include <mutex>
 #include <type_traits>
 
 #include "common.cuh"
@@ -53,69 +73,127 @@ namespace bsr {
 
 namespace gemm {
 
-constexpr int BN = 128;           // weight rows per tile (MMA M, TMEM lanes)
-constexpr int BM = 128;           // activation rows per tile (MMA N, TMEM columns)
-constexpr int KBS = 4;            // 32-blocks per stage
-constexpr int KS = 32 * KBS;      // bytes of K per stage
-constexpr int STAGES = 5;
-constexpr int TBUF = 4;           // tensor-memory ring depth (x BM columns)
-constexpr int TMEM_COLS = TBUF * BM;
-constexpr int EPI_WARPS = 16;
-constexpr int THREADS = 640;
+constexpr int BN = 128;          // weight rows per tile (MMA M, TMEM lanes)
+constexpr int KBS = 4;           // 32-blocks per stage
+constexpr int KS = 32 * KBS;     // bytes of K per stage (one 128-byte swizzle row)
 constexpr int EPI_WARP0 = 4;
-// Register split: launched with 640 x 96 = 61440 registers (the most that
-// 640 threads can hold); the control warpgroup (warps 0-3) drops to 64 and
-// the four epilogue warpgroups rise to 104: 128 x 64 + 512 x 104 = 61440.
-constexpr int LAUNCH_REGS = 96;
-constexpr int CTRL_REGS = 64;
-constexpr int EPI_REGS = 104;
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);  // 384
+// Register split: launched with 384 x 168 = 64512 registers; the control
+// warpgroup (warps 0-3) drops to 56 and the two epilogue warpgroups rise to
+// 224: 128 x 56 + 256 x 224 = 64512.
+constexpr int LAUNCH_REGS = 168;
+constexpr int CTRL_REGS = 56;
+constexpr int EPI_REGS = 224;
 static_assert(THREADS * LAUNCH_REGS <= 65536, "launch register budget");
-static_assert(128 * CTRL_REGS + (THREADS - 128) * EPI_REGS <= THREADS * LAUNCH_REGS,
+static_assert(128 * CTRL_REGS + 32 * EPI_WARPS * EPI_REGS <= THREADS * LAUNCH_REGS,
               "register split exceeds the launch allocation");
-
-constexpr int W_TILE = BN * KS;             // 16384
-constexpr int A_TILE = BM * KS;             // 16384
-constexpr int WS_TILE = BN * KBS * 4;       // 2048
-constexpr int AS_TILE = BM * KBS * 4;       // 2048
-constexpr int STAGE_BYTES = W_TILE + A_TILE + WS_TILE + AS_TILE;  // 36864
-constexpr int OFF_A = W_TILE;
-constexpr int OFF_WS = W_TILE + A_TILE;
-constexpr int OFF_AS = OFF_WS + WS_TILE;
-
+constexpr uint32_t TMEM_COLS = 512;
+// Constant operand of the bias MMA: 8 KB of 0x80 bytes read through an
+// unswizzled K-major descriptor (core matrices 8 rows x 16 bytes; 128 bytes
+// to the next one along K, 256 bytes to the next 8 rows: 256 rows x 32 bytes
+// of K span exactly 8 KB).
+constexpr int CONST_BYTES = 8192;
 constexpr uint32_t kBias = 1u << 19;  // = 32 * 128 * 128
-constexpr uint32_t kIdesc = idesc_i8(BN, BM);
-// u8 x u8 variant of the same shape, for the bias MMA
-constexpr uint32_t kIdescBias = kIdesc & ~((7u << 7) | (7u << 10));
-constexpr int CONST_TILE = BN * KS;  // 16 KB of 0x80 bytes: the bias MMA's operands
-static_assert(TBUF == KBS, "tensor-memory buffer index equals the K block index within a stage");
+constexpr size_t kSmemPerCta = 232448;  // 227 KB opt-in limit of sm_100
 
+template <int BM>
+struct Tile {
+  static constexpr int W_TILE = BN * KS;
+  static constexpr int A_TILE = BM * KS;
+  static constexpr int WS_TILE = BN * KBS * 4;
+  static constexpr int AS_TILE = BM * KBS * 4;
+  static constexpr int STAGE_BYTES = W_TILE + A_TILE + WS_TILE + AS_TILE;
+  static constexpr int OFF_A = W_TILE;
+  static constexpr int OFF_WS = W_TILE + A_TILE;
+  static constexpr int OFF_AS = OFF_WS + WS_TILE;
+  static constexpr int TBUF = (int)TMEM_COLS / BM;  // tensor-memory ring depth
+  static constexpr int COLS_W = BM / 2;             // columns per epilogue warp
+  static constexpr int CHUNKS = COLS_W / 16;        // 16-column tensor-memory loads
+  static constexpr int STAGES_FIT = (int)((kSmemPerCta - 1024 - CONST_BYTES - 512) / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT < 6 ? STAGES_FIT : 6;
+  static constexpr uint32_t IDESC = idesc_i8(BN, BM);
+  static constexpr uint32_t IDESC_BIAS = IDESC & ~((7u << 7) | (7u << 10));  // u8 x u8
+  static_assert(KBS % TBUF == 0, "buffer index pattern");
+  static_assert(BM % 32 == 0 && BM <= 256, "MMA N and the scale-prep lanes");
+  static_assert(CHUNKS >= 2, "the epilogue pipelines its tensor-memory loads over >= 2 chunks");
+  static_assert(STAGES >= 3, "shared-memory ring");
+};
+
+template <int BM>
 struct Ctrl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
-  uint64_t prep[STAGES];
-  uint64_t tfull[TBUF];
-  uint64_t tempty[TBUF];
-  int exotic[STAGES];
+  uint64_t full[Tile<BM>::STAGES];
+  uint64_t empty[Tile<BM>::STAGES];
+  uint64_t prep[Tile<BM>::STAGES];
+  uint64_t tfull[Tile<BM>::TBUF];
+  uint64_t tempty[Tile<BM>::TBUF];
+  uint64_t drain;
+  int exotic[Tile<BM>::STAGES];
   uint32_t tmem_base;
   int abort_flag;
 };
 
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + CONST_TILE + sizeof(Ctrl);
+template <int BM>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)Tile<BM>::STAGES * Tile<BM>::STAGE_BYTES + CONST_BYTES + sizeof(Ctrl<BM>);
+}
+static_assert(smem_bytes<256>() <= kSmemPerCta && smem_bytes<192>() <= kSmemPerCta &&
+                  smem_bytes<128>() <= kSmemPerCta,
+              "shared memory");
 
 __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
-template <bool DUMP>
+// Unswizzled K-major descriptor of the constant bias operand (see CONST_BYTES).
+__device__ __forceinline__ uint64_t smem_desc_const(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= (uint64_t)(128u >> 4) << 16;           // leading byte offset (next core matrix along K)
+  d |= (uint64_t)(256u >> 4) << 32;           // stride byte offset (next 8 rows)
+  d |= (uint64_t)1 << 46;                     // descriptor version (sm_100)
+  return d;                                   // layout type 0: no swizzle
+}
+
+// Ties 16 registers written by a tensor-memory load to this point of the
+// program: placed after tcgen05.wait::ld, it keeps the compiler from moving
+// their uses above the wait.
+__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[8]) {
+  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
+}
+
+// 16 lanes x 128 bits, repeated 4 times along the columns (16 columns):
+// thread t holds r[2k] = (lane t/4, column t%4 + 4k) and
+// r[2k+1] = (lane t/4 + 8, same column), k = 0..3.
+__device__ __forceinline__ void tmem_ld_16x128b_x4(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.16x128b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// Bounded wait that ignores the abort flag (used while draining).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+template <int BM, bool DUMP>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                 const __grid_constant__ CUtensorMap tm_ws, const __grid_constant__ CUtensorMap tm_as,
                 __nv_bfloat16* __restrict__ out, int32_t* __restrict__ partials, int* __restrict__ status, int m,
                 int n, int k, int n_tiles, int m_tiles, int m_fastest, long long ldo) {
+  using T = Tile<BM>;
+  constexpr int STAGES = T::STAGES;
+  constexpr int TBUF = T::TBUF;
+  constexpr int CHUNKS = T::CHUNKS;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled tiles, keeping the pointer
   // derived from the shared array so accesses stay shared-space loads
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* const_tile = smem + (size_t)STAGES * STAGE_BYTES;
-  Ctrl* ctrl = reinterpret_cast<Ctrl*>(const_tile + CONST_TILE);
+  uint8_t* const_tile = smem + (size_t)STAGES * T::STAGE_BYTES;
+  Ctrl<BM>* ctrl = reinterpret_cast<Ctrl<BM>*>(const_tile + CONST_BYTES);
   volatile int* abort_flag = &ctrl->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -127,7 +205,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctrl->full[s], 1);
-      mbar_init(&ctrl->empty[s], 2 + EPI_WARPS);  // two MMA commits + the epilogue warps
+      mbar_init(&ctrl->empty[s], 1 + EPI_WARPS);  // the MMA commit + the epilogue warps
       mbar_init(&ctrl->prep[s], 1);
       ctrl->exotic[s] = 0;
     }
@@ -135,6 +213,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&ctrl->tfull[b], 1);
       mbar_init(&ctrl->tempty[b], EPI_WARPS);
     }
+    mbar_init(&ctrl->drain, 1);
     ctrl->abort_flag = 0;
     fence_mbar_init();
   }
@@ -148,7 +227,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < CONST_TILE / 16; i += THREADS)
+  for (int i = threadIdx.x; i < CONST_BYTES / 16; i += THREADS)
     reinterpret_cast<uint4*>(const_tile)[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
   fence_proxy_async_smem();
   tc_fence_before();
@@ -172,235 +251,240 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp < EPI_WARP0) {
     setmaxnreg_dec<CTRL_REGS>();
     if (warp == 0) {
-    // ---------------------------------------------------------------- TMA
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        int n0, m0;
-        tile_coords(tile, n0, m0);
-        for (int ks = 0; ks < kstages; ++ks, ++it) {
-          const int s = it % STAGES;
-          const uint32_t r = it / STAGES;
-          if (!mbar_wait(&ctrl->empty[s], (r & 1) ^ 1, abort_flag, status, DEV_ERR_TIMEOUT_TMA)) goto tma_done;
-          uint8_t* st = smem + (size_t)s * STAGE_BYTES;
-          mbar_arrive_expect_tx(&ctrl->full[s], STAGE_BYTES);
-          tma_load_2d(st, &tm_w, &ctrl->full[s], ks * KS, n0);
-          tma_load_2d(st + OFF_A, &tm_a, &ctrl->full[s], ks * KS, m0);
-          tma_load_2d(st + OFF_WS, &tm_ws, &ctrl->full[s], ks * KBS, n0);
-          tma_load_2d(st + OFF_AS, &tm_as, &ctrl->full[s], m0, ks * KBS);
-        }
-      }
-    tma_done:;
-    }
-    } else if (warp == 1 || warp == 3) {
-    // ---------------------------------------------------------------- MMA
-    // Two issuing threads: warp 1 takes K blocks 0 and 2 of every stage,
-    // warp 3 blocks 1 and 3 (= tensor-memory buffers), so the per-block issue
-    // cost (two MMAs and a commit) is paid on two warps.
-    if (lane == 0) {
-      const uint64_t c_desc = smem_desc_k_sw128(smem_u32(const_tile));
-      const int kb0 = (warp == 1) ? 0 : 1;
-      uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-        for (int ks = 0; ks < kstages; ++ks, ++it) {
-          const int s = it % STAGES;
-          const uint32_t r = it / STAGES;
-          if (!mbar_wait(&ctrl->full[s], r & 1, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + (size_t)s * STAGE_BYTES);
-          const uint32_t b_base = a_base + OFF_A;
-#pragma unroll
-          for (int kb = kb0; kb < KBS; kb += 2) {
-            if (!mbar_wait(&ctrl->tempty[kb], it & 1, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
-            tc_fence_after();
-            // D = 2^19 (constant u8 tiles of 128s, accumulate off), then D += A x B
-            mma_i8(tmem_base + kb * BM, c_desc, c_desc, kIdescBias, 0u);
-            mma_i8(tmem_base + kb * BM, smem_desc_k_sw128(a_base + kb * 32), smem_desc_k_sw128(b_base + kb * 32),
-                   kIdesc, 1u);
-            tc_commit(&ctrl->tfull[kb]);
+      // -------------------------------------------------------------- TMA
+      if (lane == 0) {
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+          int n0, m0;
+          tile_coords(tile, n0, m0);
+          for (int ks = 0; ks < kstages; ++ks, ++it) {
+            const int s = (int)(it % STAGES);
+            const uint32_t r = it / STAGES;
+            if (!mbar_wait(&ctrl->empty[s], (r & 1) ^ 1, abort_flag, status, DEV_ERR_TIMEOUT_TMA)) goto tma_done;
+            uint8_t* st = smem + (size_t)s * T::STAGE_BYTES;
+            mbar_arrive_expect_tx(&ctrl->full[s], T::STAGE_BYTES);
+            tma_load_2d(st, &tm_w, &ctrl->full[s], ks * KS, n0);
+            tma_load_2d(st + T::OFF_A, &tm_a, &ctrl->full[s], ks * KS, m0);
+            tma_load_2d(st + T::OFF_WS, &tm_ws, &ctrl->full[s], ks * KBS, n0);
+            tma_load_2d(st + T::OFF_AS, &tm_as, &ctrl->full[s], m0, ks * KBS);
           }
-          tc_commit(&ctrl->empty[s]);
         }
+      tma_done:
+        // the copies of the last min(it, STAGES) stages issued must have
+        // landed before the CTA may exit (their phases complete on their own;
+        // after a normal run they have all completed already)
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+        for (uint32_t j = first; j < it; ++j)
+          if (!mbar_wait_drain(&ctrl->full[j % STAGES], (j / STAGES) & 1u)) break;
       }
-    mma_done:;
-    }
+    } else if (warp == 1) {
+      // -------------------------------------------------------------- MMA
+      if (lane == 0) {
+        const uint64_t c_desc = smem_desc_const(smem_u32(const_tile));
+        uint32_t it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+          for (int ks = 0; ks < kstages; ++ks, ++it) {
+            const int s = (int)(it % STAGES);
+            const uint32_t r = it / STAGES;
+            if (!mbar_wait(&ctrl->full[s], r & 1, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(smem + (size_t)s * T::STAGE_BYTES);
+            const uint32_t b_base = a_base + T::OFF_A;
+#pragma unroll
+            for (int kb = 0; kb < KBS; ++kb) {
+              const uint32_t g = it * KBS + kb;
+              const uint32_t buf = g % TBUF;
+              const uint32_t use = g / TBUF;
+              if (!mbar_wait(&ctrl->tempty[buf], use & 1u, abort_flag, status, DEV_ERR_TIMEOUT_MMA)) goto mma_done;
+              tc_fence_after();
+              // D = 2^19 (constant u8 operands of 128s, accumulate off), then D += A x B
+              mma_i8(tmem_base + buf * BM, c_desc, c_desc, T::IDESC_BIAS, 0u);
+              mma_i8(tmem_base + buf * BM, smem_desc_k_sw128(a_base + kb * 32), smem_desc_k_sw128(b_base + kb * 32),
+                     T::IDESC, 1u);
+              tc_commit(&ctrl->tfull[buf]);
+            }
+            tc_commit(&ctrl->empty[s]);
+          }
+        }
+      mma_done:
+        // every MMA issued so far (and the arrivals of its commits) has
+        // completed once this commit arrives
+        tc_commit(&ctrl->drain);
+        mbar_wait_drain(&ctrl->drain, 0u);
+      }
     } else if (warp == 2) {
-    // ---------------------------------------------------------------- scale prep
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      for (int ks = 0; ks < kstages; ++ks, ++it) {
-        const int s = it % STAGES;
-        const uint32_t r = it / STAGES;
-        if (!mbar_wait(&ctrl->full[s], r & 1, abort_flag, status, DEV_ERR_TIMEOUT_PREP)) goto prep_done;
-        uint8_t* st = smem + (size_t)s * STAGE_BYTES;
-        float4* as4 = reinterpret_cast<float4*>(st + OFF_AS);
-        float4* ws4 = reinterpret_cast<float4*>(st + OFF_WS);
-        float4 av[4], wv[4];
-        bool bad = false;
+      // -------------------------------------------------------------- scale prep
+      uint32_t it = 0;
+      for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        for (int ks = 0; ks < kstages; ++ks, ++it) {
+          const int s = (int)(it % STAGES);
+          const uint32_t r = it / STAGES;
+          if (!mbar_wait(&ctrl->full[s], r & 1, abort_flag, status, DEV_ERR_TIMEOUT_PREP)) goto prep_done;
+          uint8_t* st = smem + (size_t)s * T::STAGE_BYTES;
+          float* wsf = reinterpret_cast<float*>(st + T::OFF_WS);  // [n][kb] as loaded
+          float* asf = reinterpret_cast<float*>(st + T::OFF_AS);  // [kb][m] as loaded
+          // pass 1: is every scale of the stage inside the fast path's window?
+          bool bad = false;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          av[j] = as4[j * 32 + lane];
-          bad |= !(av[j].x < 0x1p79f) | !(av[j].y < 0x1p79f) | !(av[j].z < 0x1p79f) | !(av[j].w < 0x1p79f);
-          wv[j] = ws4[j * 32 + lane];
-          const float w4[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float aw = fabsf(w4[t]);
+          for (int i = 0; i < (BN * KBS) / 32; ++i) {
+            const float aw = fabsf(wsf[i * 32 + lane]);
             bad |= !((aw == 0.0f) | ((aw >= 0x1p-77f) & (aw < 0x1p28f)));
           }
-        }
-        const bool exotic = __any_sync(0xFFFFFFFFu, bad);
-        // a_scale * 2^49 and W = w_scale * 2^100 (exact inside the window;
-        // an exotic stage keeps the scales as loaded)
-        const float fa = exotic ? 1.0f : 0x1p49f;
-        const float fw = exotic ? 1.0f : 0x1p100f;
-        __syncwarp();
-        // Rewrite both scale tiles in the order the epilogue reads them.
-        // Activation scales [kb][m], m = 32h + r + 4k  ->  [kb][h][r][k]:
-        // lane L holds m = 4L..4L+3 of every kb (h = L/8, k = L%8, r = e).
-        // Weight scales [n][kb], n = 32q + l + 8i  ->  [kb][q][l][i]: lane L
-        // holds row n = 32j + L (q = j, l = L%8, i = L/8) for all four kb.
-        float* asf = reinterpret_cast<float*>(st + OFF_AS);
-        float* wsf = reinterpret_cast<float*>(st + OFF_WS);
+#pragma unroll 4
+          for (int i = 0; i < (BM * KBS) / 32; ++i) bad |= !(asf[i * 32 + lane] < 0x1p79f);
+          const bool exotic = __any_sync(0xFFFFFFFFu, bad);
+          const float fa = exotic ? 1.0f : 0x1p49f;
+          const float fw = exotic ? 1.0f : 0x1p100f;
+          // pass 2: rewrite both tiles in the order the epilogue reads them.
+          // Weight scales [n][kb], n = 32q + 8i + l  ->  [kb][q][l][i]: lane L
+          // holds the four kb of row 32q + L (l = L%8, i = L/8).
+          float4 wv[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float a4[4] = {av[j].x, av[j].y, av[j].z, av[j].w};
-          const float w4[4] = {wv[j].x, wv[j].y, wv[j].z, wv[j].w};
+          for (int q = 0; q < 4; ++q) wv[q] = reinterpret_cast<const float4*>(wsf)[q * 32 + lane];
+          __syncwarp();
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            asf[j * BM + (lane >> 3) * 32 + e * 8 + (lane & 7)] = a4[e] * fa;
-            wsf[e * BN + j * 32 + (lane & 7) * 4 + (lane >> 3)] = w4[e] * fw;
+          for (int q = 0; q < 4; ++q) {
+            const float w4[4] = {wv[q].x, wv[q].y, wv[q].z, wv[q].w};
+#pragma unroll
+            for (int kb = 0; kb < KBS; ++kb) wsf[kb * BN + q * 32 + (lane & 7) * 4 + (lane >> 3)] = w4[kb] * fw;
+          }
+          // Activation scales [kb][m], m = 16g + 4j + r  ->  [kb][g][r][j]
+          // (g = 16-column group, r = t%4 of the epilogue thread, j = its
+          // column index within the group): a permutation inside each group.
+          // Lane L takes m = 32G + L, i.e. group 2G + L/16, j = (L/4)%4.
+#pragma unroll 1
+          for (int kb = 0; kb < KBS; ++kb) {
+            float av[BM / 32];
+#pragma unroll
+            for (int g = 0; g < BM / 32; ++g) av[g] = asf[kb * BM + g * 32 + lane];
+            __syncwarp();
+            const int dst = (lane >> 4) * 16 + (lane & 3) * 4 + ((lane >> 2) & 3);
+#pragma unroll
+            for (int g = 0; g < BM / 32; ++g) asf[kb * BM + g * 32 + dst] = av[g] * fa;
+          }
+          // the rewritten bytes are overwritten later by TMA (async proxy)
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ctrl->exotic[s] = exotic ? 1 : 0;
+            mbar_arrive(&ctrl->prep[s]);
           }
         }
-        if (lane == 0) ctrl->exotic[s] = exotic ? 1 : 0;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ctrl->prep[s]);
       }
-    }
     prep_done:;
     }
   } else {
     setmaxnreg_inc<EPI_REGS>();
-    // ---------------------------------------------------------------- epilogue
-    // Warp (quarter q, column slice h) owns tensor-memory lanes 32q..32q+31
-    // (weight rows) and columns 32h..32h+31 (activation rows), read per block
-    // with two 16x128b.x8 loads (lanes 32q..+15 and 32q+16..+31): thread t
-    // holds weight rows 32q + t/4 + 8i (i = 0..3) and activation columns
-    // 32h + t%4 + 4k (k = 0..7).  Registers r[2k], r[2k+1] of one load are
-    // rows (t/4, t/4 + 8) at the same column: the operand pair of one packed
-    // FMA.  Per block a thread needs 4 weight scales (one 16-byte load) and
-    // 8 activation scales (two), from the tiles the prep warp rewrote.
-    // A warp hands its buffer back as soon as its loads have landed and then
-    // rescales from registers; four warps per scheduler hide each other's
-    // load latency.
+    // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int h = (warp - EPI_WARP0) >> 2;
     const int l8 = lane >> 2;
     const int c4 = lane & 3;
-    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 32);
+    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * T::COLS_W);
     const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const uint32_t smem_base = smem_u32(smem);
-    const uint32_t ws_off = OFF_WS + (uint32_t)(q * 32 + l8 * 4) * 4u;  // + kb*BN*4
-    const uint32_t as_off = OFF_AS + (uint32_t)(h * 32 + c4 * 8) * 4u;  // + kb*BM*4
+    const uint32_t ws_off = T::OFF_WS + (uint32_t)(q * 32 + l8 * 4) * 4u;                // + kb*BN*4
+    const uint32_t as_off = T::OFF_AS + (uint32_t)(h * T::COLS_W + c4 * 4) * 4u;         // + kb*BM*4 + c*64
 
     // open the tensor-memory ring
-    mbar_arrive_lane0(&ctrl->tempty[0], lane);
-    mbar_arrive_lane0(&ctrl->tempty[1], lane);
-    mbar_arrive_lane0(&ctrl->tempty[2], lane);
-    mbar_arrive_lane0(&ctrl->tempty[3], lane);
-
-    float2 acc[2][8];  // acc[j][k] = rows (2j, 2j+1) of this thread's four, column k
-    uint32_t r0[16], r1[16];
-
-    auto dump = [&](int n0, int m0, int b) {
-      if constexpr (DUMP) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int nn = n0 + q * 32 + l8 + 8 * i;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const int mm = m0 + h * 32 + c4 + 4 * k;
-            const uint32_t v = (i < 2) ? r0[2 * k + (i & 1)] : r1[2 * k + (i & 1)];
-            if (nn < n && mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)v - (int)kBias;
-          }
-        }
-      }
-    };
+    for (int b = 0; b < TBUF; ++b) mbar_arrive_lane0(&ctrl->tempty[b], lane);
 
-    // Stage sequence of this CTA: stage counter itg (tiles x K stages), ring
-    // slot itg % STAGES; within a stage the four K blocks are unrolled, block
-    // kb in tensor-memory buffer kb (phase itg & 1).
+    float2 acc[CHUNKS][2][4];  // acc[c][j][k]: rows (l8 + 16j, l8 + 16j + 8), column 16c + c4 + 4k
+    uint32_t ra[2][8], rb[2][8];
+
     const int total_st = my_tiles * kstages;
     int tile = blockIdx.x, n0 = 0, m0 = 0, kst = 0;
     tile_coords(tile, n0, m0);
     uint32_t st_addr = smem_base;
     uint32_t itg = 0;
 
-    // One K block: scales, partials, buffer release, rescale.  The choice of
-    // the exotic path is a template parameter, so a stage runs one of two
-    // fully unrolled code paths with no branch inside.
-    auto sub = [&](auto kbc, auto exc) -> bool {
-      constexpr int kb = decltype(kbc)::value;
-      constexpr bool EXO = decltype(exc)::value;
-      const float4 W4 = lds_f32x4(st_addr + ws_off + (uint32_t)kb * (BN * 4u));
-      const float4 A0 = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u));
-      const float4 A1 = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u) + 16u);
-      if (!mbar_wait(&ctrl->tfull[kb], itg & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
-      tc_fence_after();
-      tmem_ld_16x128b_x8(tl + kb * BM, r0);
-      tmem_ld_16x128b_x8(tl + kb * BM + (16u << 16), r1);
-      tc_wait_ld();
-      tc_fence_before();
-      mbar_arrive_lane0(&ctrl->tempty[kb], lane);
-      const float av[8] = {A0.x, A0.y, A0.z, A0.w, A1.x, A1.y, A1.z, A1.w};
-      const float2 Wp[2] = {make_float2(W4.x, W4.y), make_float2(W4.z, W4.w)};
-      if constexpr (!EXO) {
-        const float2 Cp[2] = {make_float2(-(W4.x * 0x1p-130f), -(W4.y * 0x1p-130f)),
-                              make_float2(-(W4.z * 0x1p-130f), -(W4.w * 0x1p-130f))};
+    auto dump = [&](int c, int b, const uint32_t (&x)[8], const uint32_t (&y)[8]) {
+      if constexpr (DUMP) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float2 u0 = __ffma2_rn(f2(r0[2 * k], r0[2 * k + 1]), Wp[0], Cp[0]);
-          const float2 u1 = __ffma2_rn(f2(r1[2 * k], r1[2 * k + 1]), Wp[1], Cp[1]);
-          acc[0][k] = __ffma2_rn(u0, make_float2(av[k], av[k]), acc[0][k]);
-          acc[1][k] = __ffma2_rn(u1, make_float2(av[k], av[k]), acc[1][k]);
-        }
-      } else {
+        for (int i = 0; i < 4; ++i) {
+          const int nn = n0 + q * 32 + l8 + 8 * i;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const uint32_t* rr = j ? r1 : r0;
-            const float ux = __fmul_rn(__int2float_rn((int)rr[2 * k] - (int)kBias), j ? W4.z : W4.x);
-            const float uy = __fmul_rn(__int2float_rn((int)rr[2 * k + 1] - (int)kBias), j ? W4.w : W4.y);
-            acc[j][k].x = __fmaf_rn(ux, av[k], acc[j][k].x);
-            acc[j][k].y = __fmaf_rn(uy, av[k], acc[j][k].y);
+          for (int kk = 0; kk < 4; ++kk) {
+            const int mm = m0 + h * T::COLS_W + c * 16 + c4 + 4 * kk;
+            const uint32_t v = (i < 2) ? x[2 * kk + (i & 1)] : y[2 * kk + (i & 1)];
+            if (nn < n && mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)v - (int)kBias;
           }
         }
       }
-      dump(n0, m0, kst * KBS + kb);
-      if (kb == KBS - 1) {
-        mbar_arrive_lane0(&ctrl->empty[(int)(itg % STAGES)], lane);
-        if (++kst == kstages) {
-          // tile end: write BF16 out[m][n]; the tile origin passes through a
-          // volatile move so the store addresses are formed here only
-          int nr, mr;
-          asm volatile("mov.b32 %0, %1;" : "=r"(nr) : "r"(n0 + q * 32 + l8));
-          asm volatile("mov.b32 %0, %1;" : "=r"(mr) : "r"(m0 + h * 32 + c4));
+    };
+
+    // One K block: weight scales, pipelined chunk loads, buffer release,
+    // rescale.  kb and the exotic choice are template parameters, so a stage
+    // runs one of two fully unrolled code paths with no branch inside.
+    auto block = [&](auto kbc, auto exc) -> bool {
+      constexpr int kb = decltype(kbc)::value;
+      constexpr bool EXO = decltype(exc)::value;
+      const uint32_t g = itg * KBS + kb;
+      const uint32_t buf = (uint32_t)(kb % TBUF);  // TBUF divides KBS*itg
+      const uint32_t par = (g / TBUF) & 1u;
+      const float4 W4 = lds_f32x4(st_addr + ws_off + (uint32_t)kb * (BN * 4u));
+      const float2 Wp0 = make_float2(W4.x, W4.y), Wp1 = make_float2(W4.z, W4.w);
+      float2 Cp0, Cp1;
+      if constexpr (!EXO) {
+        Cp0 = __fmul2_rn(Wp0, make_float2(-0x1p-130f, -0x1p-130f));
+        Cp1 = __fmul2_rn(Wp1, make_float2(-0x1p-130f, -0x1p-130f));
+      }
+      if (!mbar_wait(&ctrl->tfull[buf], par, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
+      tc_fence_after();
+      const uint32_t tb = tl + buf * BM;
+      tmem_ld_16x128b_x4(tb, ra[0]);
+      tmem_ld_16x128b_x4(tb + (16u << 16), rb[0]);
+      tc_wait_ld();
+      regs_after_wait(ra[0]);
+      regs_after_wait(rb[0]);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int nn = nr + 8 * i;
-            if (nn < n) {
+      for (int c = 0; c < CHUNKS; ++c) {
+        const int cur = c & 1;
+        // the fast path loads the next chunk while it rescales this one; the
+        // exotic path (rare) loads it afterwards and keeps one buffer live
+        if (!EXO && c + 1 < CHUNKS) {
+          tmem_ld_16x128b_x4(tb + 16u * (c + 1), ra[cur ^ 1]);
+          tmem_ld_16x128b_x4(tb + 16u * (c + 1) + (16u << 16), rb[cur ^ 1]);
+        }
+        const float4 A0 = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u) + (uint32_t)c * 64u);
+        const float av[4] = {A0.x, A0.y, A0.z, A0.w};
+        dump(c, (kst * KBS) + kb, ra[cur], rb[cur]);
+        if constexpr (!EXO) {
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                const int mm = mr + 4 * k;
-                const float v = (i & 1) ? acc[i >> 1][k].y : acc[i >> 1][k].x;
-                if (mm < m) out[(size_t)mm * (size_t)ldo + nn] = __float2bfloat16_rn(v);
-              }
+          for (int kk = 0; kk < 4; ++kk) {
+            const float2 u0 = __ffma2_rn(f2(ra[cur][2 * kk], ra[cur][2 * kk + 1]), Wp0, Cp0);
+            const float2 u1 = __ffma2_rn(f2(rb[cur][2 * kk], rb[cur][2 * kk + 1]), Wp1, Cp1);
+            const float2 ap = make_float2(av[kk], av[kk]);
+            acc[c][0][kk] = __ffma2_rn(u0, ap, acc[c][0][kk]);
+            acc[c][1][kk] = __ffma2_rn(u1, ap, acc[c][1][kk]);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const uint32_t* rr = j ? rb[cur] : ra[cur];
+              const float ux = __fmul_rn(__int2float_rn((int)rr[2 * kk] - (int)kBias), j ? W4.z : W4.x);
+              const float uy = __fmul_rn(__int2float_rn((int)rr[2 * kk + 1] - (int)kBias), j ? W4.w : W4.y);
+              acc[c][j][kk].x = __fmaf_rn(ux, av[kk], acc[c][j][kk].x);
+              acc[c][j][kk].y = __fmaf_rn(uy, av[kk], acc[c][j][kk].y);
             }
           }
-          kst = 0;
-          tile += gridDim.x;
-          tile_coords(tile, n0, m0);
+        }
+        if (c + 1 < CHUNKS) {
+          if (EXO) {
+            tmem_ld_16x128b_x4(tb + 16u * (c + 1), ra[cur ^ 1]);
+            tmem_ld_16x128b_x4(tb + 16u * (c + 1) + (16u << 16), rb[cur ^ 1]);
+          }
+          tc_wait_ld();
+          regs_after_wait(ra[cur ^ 1]);
+          regs_after_wait(rb[cur ^ 1]);
+          if (c + 2 == CHUNKS) {
+            // the last chunk is in registers: hand the buffer back to the MMA
+            tc_fence_before();
+            mbar_arrive_lane0(&ctrl->tempty[buf], lane);
+          }
         }
       }
       return true;
@@ -410,13 +494,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (; ok && itg < (uint32_t)total_st; ++itg) {
       const int s = (int)(itg % STAGES);
       if (!mbar_wait(&ctrl->prep[s], (itg / STAGES) & 1u, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) break;
-      st_addr = smem_base + (uint32_t)s * STAGE_BYTES;
+      st_addr = smem_base + (uint32_t)s * T::STAGE_BYTES;
       const int exotic = ctrl->exotic[s];
       if (kst == 0) {
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
+        for (int c = 0; c < CHUNKS; ++c)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) acc[j][k] = make_float2(0.0f, 0.0f);
+          for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) acc[c][j][kk] = make_float2(0.0f, 0.0f);
       }
       using K0 = std::integral_constant<int, 0>;
       using K1 = std::integral_constant<int, 1>;
@@ -424,10 +510,40 @@ __global__ void __launch_bounds__(THREADS, 1)
       using K3 = std::integral_constant<int, 3>;
       if (!exotic) {
         const std::false_type fast;
-        ok = sub(K0{}, fast) && sub(K1{}, fast) && sub(K2{}, fast) && sub(K3{}, fast);
+        ok = block(K0{}, fast) && block(K1{}, fast) && block(K2{}, fast) && block(K3{}, fast);
       } else {
         const std::true_type slow;
-        ok = sub(K0{}, slow) && sub(K1{}, slow) && sub(K2{}, slow) && sub(K3{}, slow);
+        ok = block(K0{}, slow) && block(K1{}, slow) && block(K2{}, slow) && block(K3{}, slow);
+      }
+      if (!ok) break;
+      // this stage's scales are no longer read
+      mbar_arrive_lane0(&ctrl->empty[s], lane);
+      if (++kst == kstages) {
+        // tile end: write BF16 out[m][n], one activation row (4 weight rows
+        // of it) at a time; the row pointer advances by a volatile add so the
+        // compiler does not form all the store addresses at once
+        const int nr = n0 + q * 32 + l8;
+        const int mr = m0 + h * T::COLS_W + c4;
+        __nv_bfloat16* p = out + (size_t)mr * (size_t)ldo + nr;
+        const long long step = 4 * ldo;
+#pragma unroll
+        for (int c = 0; c < CHUNKS; ++c) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int mm = mr + 16 * c + 4 * kk;
+            if (mm < m) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float v = (i & 1) ? acc[c][i >> 1][kk].y : acc[c][i >> 1][kk].x;
+                if (nr + 8 * i < n) p[8 * i] = __float2bfloat16_rn(v);
+              }
+            }
+            asm volatile("add.s64 %0, %0, %1;" : "+l"(p) : "l"(step * 2));
+          }
+        }
+        kst = 0;
+        tile += gridDim.x;
+        tile_coords(tile, n0, m0);
       }
     }
   }
@@ -438,15 +554,99 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// Shared-memory opt-in per device and kernel variant, made once under a lock.
+std::mutex g_optin_mu;
+bool g_optin[64][6] = {};
+
+template <int BM, bool DUMP>
+cudaError_t optin_variant(int dev) {
+  const int slot = (BM == 128 ? 0 : BM == 192 ? 2 : 4) + (DUMP ? 1 : 0);
+  if (g_optin[dev][slot]) return cudaSuccess;
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, gemm_kernel<BM, DUMP>);
+  if (e != cudaSuccess) return e;
+  // the register split assumes every thread starts with LAUNCH_REGS registers
+  if (fa.numRegs < LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(gemm_kernel<BM, DUMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<BM>());
+  if (e != cudaSuccess) return e;
+  g_optin[dev][slot] = true;
+  return cudaSuccess;
+}
+
+template <int BM>
+cudaError_t optin(int dev, bool partials) {
+  return partials ? optin_variant<BM, true>(dev) : optin_variant<BM, false>(dev);
+}
+
+template <int BM>
+void launch_bm(const GemmMaps& maps, __nv_bfloat16* out, int32_t* partials, int* status, int m, int n, int k,
+               long long ldo, cudaStream_t stream, int grid, int n_tiles, int m_tiles, int m_fastest) {
+  if (partials)
+    gemm_kernel<BM, true><<<grid, THREADS, smem_bytes<BM>(), stream>>>(
+        maps.w, maps.a, maps.ws, maps.as, out, partials, status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
+  else
+    gemm_kernel<BM, false><<<grid, THREADS, smem_bytes<BM>(), stream>>>(
+        maps.w, maps.a, maps.ws, maps.as, out, nullptr, status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
+}
+
+// Relative epilogue throughput per element of the tile widths, measured on
+// B200 from whole-kernel times of the three widths on the 2048 x 14336 x
+// 4096, 8192 x 4096 x 14336 and 4095 x 8192 x 8192 projections (they agree
+// within 2%): 192 rows give each thread 96 columns with no register spills;
+// 256 rows need more registers than the epilogue warps hold.
+constexpr double kRate128 = 1.0, kRate192 = 1.10, kRate256 = 0.945;
+
 }  // namespace gemm
 
-size_t gemm_smem_bytes() { return gemm::SMEM_BYTES; }
+int gemm_block_m(long long m, long long n, int num_sms) {
+  // M <= 128: one activation tile.  Otherwise the width with the least
+  // estimated time: whole waves of persistent tiles x tile width / rate.
+  if (m <= 128) return 128;
+  const long long nt = (n + gemm::BN - 1) / gemm::BN;
+  const int widths[3] = {256, 192, 128};
+  const double rates[3] = {gemm::kRate256, gemm::kRate192, gemm::kRate128};
+  int best = 256;
+  double best_t = 0.0;
+  for (int i = 0; i < 3; ++i) {
+    const long long tiles = nt * ((m + widths[i] - 1) / widths[i]);
+    const long long waves = (tiles + num_sms - 1) / num_sms;
+    const double t = (double)waves * widths[i] / rates[i];
+    if (i == 0 || t < best_t * (1.0 - 1e-9)) {
+      best = widths[i];
+      best_t = t;
+    }
+  }
+  return best;
+}
+
+long long gemm_tiles(long long m, long long n, int num_sms) {
+  const long long bm = gemm_block_m(m, n, num_sms);
+  return ((n + gemm::BN - 1) / gemm::BN) * ((m + bm - 1) / bm);
+}
+
+size_t gemm_smem_bytes() { return gemm::smem_bytes<256>(); }
+
+cudaError_t gemm_prepare_device(bool partials, int bm) {
+  using namespace gemm;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_optin_mu);
+  switch (bm) {
+    case 128: return optin<128>(dev, partials);
+    case 192: return optin<192>(dev, partials);
+    case 256: return optin<256>(dev, partials);
+    default: return cudaErrorInvalidValue;
+  }
+}
 
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
-                        long long ldo, cudaStream_t stream, int num_sms, int max_ctas) {
+                        int bm, long long ldo, cudaStream_t stream, int num_sms, int max_ctas) {
   using namespace gemm;
   const int n_tiles = (n + BN - 1) / BN;
-  const int m_tiles = (m + BM - 1) / BM;
+  const int m_tiles = (m + bm - 1) / bm;
   const int tiles = n_tiles * m_tiles;
   // persistent CTAs: one per SM, or fewer when the caller shares the GPU
   // between concurrent launches (max_ctas)
@@ -455,30 +655,12 @@ cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, 
   // Sweep the smaller operand fastest so that it stays resident in L2 while
   // the larger one streams through once.
   const int m_fastest = ((long long)m <= (long long)n) ? 1 : 0;
-  // the shared-memory opt-in is set once per device and kernel variant
-  static bool granted[64][2] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (partials) {
-    if (!granted[dev][1]) {
-      e = cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      granted[dev][1] = true;
-    }
-    gemm_kernel<true><<<grid, THREADS, SMEM_BYTES, stream>>>(maps.w, maps.a, maps.ws, maps.as,
-                                                             reinterpret_cast<__nv_bfloat16*>(out), partials,
-                                                             status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
-  } else {
-    if (!granted[dev][0]) {
-      e = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-      if (e != cudaSuccess) return e;
-      granted[dev][0] = true;
-    }
-    gemm_kernel<false><<<grid, THREADS, SMEM_BYTES, stream>>>(maps.w, maps.a, maps.ws, maps.as,
-                                                              reinterpret_cast<__nv_bfloat16*>(out), nullptr,
-                                                              status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
+  __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(out);
+  switch (bm) {
+    case 128: launch_bm<128>(maps, o, partials, status, m, n, k, ldo, stream, grid, n_tiles, m_tiles, m_fastest); break;
+    case 192: launch_bm<192>(maps, o, partials, status, m, n, k, ldo, stream, grid, n_tiles, m_tiles, m_fastest); break;
+    case 256: launch_bm<256>(maps, o, partials, status, m, n, k, ldo, stream, grid, n_tiles, m_tiles, m_fastest); break;
+    default: return cudaErrorInvalidValue;
   }
   return cudaGetLastError();
 }

@@ -8,12 +8,19 @@
 
 namespace bsr {
 
+// Tensor maps of one GEMM launch.  BM = gemm_block_m(M, N, SMs) activation
+// rows per tile (128, 192 or 256), 128 weight rows, 4 K blocks per stage.
 struct GemmMaps {
-  CUtensorMap w;   // W_i8 [N, K] int8, box 128 x 128 B, 128-byte swizzle
-  CUtensorMap a;   // a_i8 [M, K] int8, box 128 x 128 B, 128-byte swizzle
-  CUtensorMap ws;  // W_scale [N, K/32] f32, box 128 x 4
-  CUtensorMap as;  // a_scale_t [K/32, ld] f32 (dims K/32 x M), box 4 x 128
+  CUtensorMap w;   // W_i8 [N, K] int8, box 128 rows x 128 B, 128-byte swizzle
+  CUtensorMap a;   // a_i8 [M, K] int8, box BM rows x 128 B, 128-byte swizzle
+  CUtensorMap ws;  // W_scale [N, K/32] f32, box 128 rows x 4
+  CUtensorMap as;  // a_scale_t [K/32, ld] f32 (dims K/32 x M), box 4 rows x BM
 };
+constexpr int kGemmBoxK = 128;  // bytes of K per stage
+constexpr int kGemmBoxW = 128;  // weight rows per tile
+constexpr int kGemmBoxKB = 4;   // 32-blocks per stage
+int gemm_block_m(long long m, long long n, int num_sms);
+long long gemm_tiles(long long m, long long n, int num_sms);
 
 cudaError_t launch_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2, int8_t* w_i8,
                              float* w_scale, long long n, long long k, cudaStream_t stream, int num_sms);
@@ -38,11 +45,15 @@ cudaError_t launch_decode_stacked(const uint16_t* a, const DecodeSegs& segs, uin
                                   int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
                                   int num_sms);
 size_t gemm_smem_bytes();
+// Shared-memory opt-in of the kernel variant with tile width bm (with or
+// without the partials dump), once per device, thread-safe.  Fails if the
+// kernel was not built with the register count its register split assumes.
+cudaError_t gemm_prepare_device(bool partials, int bm);
 // out row stride ldo (elements) >= n: the output may be a column slice of a
 // wider matrix.  max_ctas > 0 caps the persistent grid (to share the GPU
 // between concurrent launches).
 cudaError_t launch_gemm(const GemmMaps& maps, uint16_t* out, int32_t* partials, int* status, int m, int n, int k,
-                        long long ldo, cudaStream_t stream, int num_sms, int max_ctas = 0);
+                        int bm, long long ldo, cudaStream_t stream, int num_sms, int max_ctas = 0);
 
 // SiLU.mul: x = bf16(silu(g) * u) (x, g, u [M, K] BF16), and the fused
 // quantiser requant_a(bf16(silu(g) * u)) into the requant_a layout.

@@ -351,6 +351,27 @@ bsr_status launched(cudaError_t e, const char* what) {
 }
 
 }  // namespace
+
+// Row quantiser launch (8 rows per CTA, programmatic stream serialisation so
+// a dependent kernel may start its prologue early).
+cudaError_t launch_nvfp4_quant_rows(const uint16_t* a, uint8_t* a_packed, uint8_t* a_e4m3, float* a_scale2, int m,
+                                    int k, cudaStream_t stream, int num_sms) {
+  long long grid = (m + 7) / 8;  // 8 rows (warps) per CTA
+  if (grid > 8LL * num_sms) grid = 8LL * num_sms;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(256);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, nvfp4_quant_rows_kernel, a, a_packed, a_e4m3, a_scale2, m, k);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  return e;
+}
+
 }  // namespace bsr
 
 extern "C" {
@@ -366,19 +387,8 @@ bsr_status bsr_nvfp4_quant_rows(const uint16_t* a, uint8_t* a_packed, uint8_t* a
   bsr::Dev d;
   int dev = 0;
   if ((st = bsr::query_device(d, dev)) != BSR_OK) return st;
-  long long grid = (m + 7) / 8;  // 8 rows (warps) per CTA
-  if (grid > 8LL * d.num_sms) grid = 8LL * d.num_sms;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(256);
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, bsr::nvfp4_quant_rows_kernel, a, a_packed, a_e4m3, a_scale2, (int)m, (int)k);
-  if (e == cudaSuccess) e = cudaGetLastError();
+  const cudaError_t e = bsr::launch_nvfp4_quant_rows(a, a_packed, a_e4m3, a_scale2, (int)m, (int)k,
+                                                     reinterpret_cast<cudaStream_t>(stream), d.num_sms);
   return bsr::launched(e, "nvfp4 row quantiser launch");
 }
 

@@ -46,6 +46,11 @@
 namespace bsr {
 // Records the message bsr_last_error() returns on this thread (api.cu).
 bsr_status report(bsr_status st, const char* fmt, ...);
+// Device address of the library's status word on the current device (api.cu).
+bsr_status library_status_word(int** out);
+// The NVFP4 row quantiser's launch (w4a4.cu).
+cudaError_t launch_nvfp4_quant_rows(const uint16_t* a, uint8_t* a_packed, uint8_t* a_e4m3, float* a_scale2, int m,
+                                    int k, cudaStream_t stream, int num_sms);
 }  // namespace bsr
 
 namespace bsr {
@@ -390,6 +395,67 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 long long sf_blocked_bytes(long long rows, long long k) { return (rows + 127) / 128 * (k / 64) * 512; }
 
+cudaError_t launch_sf_blocked(const uint8_t* e4m3, uint8_t* blocked, long long rows, long long k, cudaStream_t stream,
+                              int num_sms) {
+  const long long words = sf_blocked_bytes(rows, k) / 4;
+  long long grid = (words + 255) / 256;
+  if (grid > 8LL * num_sms) grid = 8LL * num_sms;
+  sf_blocked_kernel<<<(unsigned)grid, 256, 0, stream>>>(e4m3, reinterpret_cast<uint32_t*>(blocked), (int)rows,
+                                                        (int)k, words);
+  return cudaGetLastError();
+}
+
+// Everything a GEMM launch needs, prepared (and every check done) before
+// anything is queued.
+struct GemmLaunch {
+  CUtensorMap tm_a, tm_w;
+  int grid, m_tiles, n_tiles, m_fastest, vec_store;
+};
+
+bsr_status prepare_gemm(GemmLaunch& g, const uint8_t* a_packed, const uint8_t* w_packed, long long m, long long n,
+                        long long k, int num_sms) {
+  bsr_status st;
+  if ((st = encode_fp4_map(&g.tm_a, a_packed, m, k, "a_packed")) != BSR_OK) return st;
+  if ((st = encode_fp4_map(&g.tm_w, w_packed, n, k, "w_packed")) != BSR_OK) return st;
+  g.m_tiles = (int)((m + BM - 1) / BM);
+  g.n_tiles = (int)((n + BN - 1) / BN);
+  const long long tiles = (long long)g.m_tiles * g.n_tiles;
+  if (tiles > 0x7FFFFFFFLL) return report(BSR_EINVAL, "too many tiles");
+  g.grid = (int)(tiles < num_sms ? tiles : num_sms);
+  // sweep the smaller operand fastest so it stays in L2 while the larger one
+  // streams through once
+  g.m_fastest = m <= n ? 1 : 0;
+  g.vec_store = n % 8 == 0 ? 1 : 0;
+  return BSR_OK;
+}
+
+cudaError_t launch_prepared(const GemmLaunch& g, const uint8_t* a_sf, const uint8_t* w_sf, const float* a_scale2,
+                            float scale2, uint16_t* out, int* status, long long m, long long n, long long k,
+                            cudaStream_t stream) {
+  w4a4_gemm_kernel<<<g.grid, THREADS, SMEM_BYTES, stream>>>(
+      g.tm_a, g.tm_w, a_sf, w_sf, a_scale2, scale2, reinterpret_cast<__nv_bfloat16*>(out), status, (int)m, (int)n,
+      (int)k, g.m_tiles, g.n_tiles, g.m_fastest, g.vec_store);
+  return cudaGetLastError();
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Scratch of the composite entry: packed codes, E4M3 bytes, blocked scales,
+// row scales, each 256-byte aligned.
+struct ProjScratch {
+  size_t packed, e4m3, blocked, scale2, total;
+};
+
+ProjScratch proj_scratch(long long m, long long k) {
+  ProjScratch p;
+  p.packed = 0;
+  p.e4m3 = align256((size_t)m * (size_t)(k / 2));
+  p.blocked = p.e4m3 + align256((size_t)m * (size_t)(k / 16));
+  p.scale2 = p.blocked + align256((size_t)sf_blocked_bytes(m, k));
+  p.total = p.scale2 + align256((size_t)m * 4);
+  return p;
+}
+
 }  // namespace w4gemm
 }  // namespace bsr
 
@@ -413,12 +479,7 @@ bsr_status bsr_nvfp4_sf_blocked(const uint8_t* e4m3, uint8_t* blocked, int64_t r
   int dev = 0;
   bsr_status st = query_device(d, dev);
   if (st != BSR_OK) return st;
-  const long long words = sf_blocked_bytes(rows, k) / 4;
-  long long grid = (words + 255) / 256;
-  if (grid > 8LL * d.num_sms) grid = 8LL * d.num_sms;
-  sf_blocked_kernel<<<(unsigned)grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      e4m3, reinterpret_cast<uint32_t*>(blocked), (int)rows, (int)k, words);
-  const cudaError_t e = cudaGetLastError();
+  const cudaError_t e = launch_sf_blocked(e4m3, blocked, rows, k, reinterpret_cast<cudaStream_t>(stream), d.num_sms);
   if (e != cudaSuccess) return bsr::report(BSR_ECUDA, "scale relayout launch: %s", cudaGetErrorString(e));
   return bsr::report(BSR_OK, "");
 }
@@ -441,22 +502,58 @@ bsr_status bsr_w4a4_gemm(const uint8_t* a_packed, const uint8_t* a_sf_blocked, c
   int dev = 0;
   bsr_status st = query_device(d, dev);
   if (st != BSR_OK) return st;
-  CUtensorMap tm_a, tm_w;
-  if ((st = encode_fp4_map(&tm_a, a_packed, m, k, "a_packed")) != BSR_OK) return st;
-  if ((st = encode_fp4_map(&tm_w, w_packed, n, k, "w_packed")) != BSR_OK) return st;
-  const int m_tiles = (int)((m + BM - 1) / BM);
-  const int n_tiles = (int)((n + BN - 1) / BN);
-  const long long tiles = (long long)m_tiles * n_tiles;
-  if (tiles > 0x7FFFFFFFLL) return bsr::report(BSR_EINVAL, "too many tiles");
-  const int grid = (int)(tiles < d.num_sms ? tiles : d.num_sms);
-  // sweep the smaller operand fastest so it stays in L2 while the larger one
-  // streams through once
-  const int m_fastest = m <= n ? 1 : 0;
-  w4a4_gemm_kernel<<<grid, THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
-      tm_a, tm_w, a_sf_blocked, w_sf_blocked, a_scale2, scale2, reinterpret_cast<__nv_bfloat16*>(out), status_dev,
-      (int)m, (int)n, (int)k, m_tiles, n_tiles, m_fastest, n % 8 == 0 ? 1 : 0);
-  const cudaError_t e = cudaGetLastError();
+  GemmLaunch g;
+  if ((st = prepare_gemm(g, a_packed, w_packed, m, n, k, d.num_sms)) != BSR_OK) return st;
+  const cudaError_t e = launch_prepared(g, a_sf_blocked, w_sf_blocked, a_scale2, scale2, out, status_dev, m, n, k,
+                                        reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return bsr::report(BSR_ECUDA, "w4a4 GEMM launch: %s", cudaGetErrorString(e));
+  return bsr::report(BSR_OK, "");
+}
+
+size_t bsr_w4a4_proj_scratch_bytes(int64_t m, int64_t k) {
+  using namespace bsr::w4gemm;
+  if (m <= 0 || m > BSR_MAX_DIM || k <= 0 || k > BSR_MAX_DIM || k % KE != 0) return 0;
+  return proj_scratch(m, k).total;
+}
+
+bsr_status bsr_w4a4_proj(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_sf_blocked, float scale2,
+                         uint16_t* out, int64_t m, int64_t n, int64_t k, void* scratch, size_t scratch_bytes,
+                         void* stream) {
+  using namespace bsr::w4gemm;
+  if (m < 0 || m > BSR_MAX_DIM || n < 0 || n > BSR_MAX_DIM || k < 0 || k > BSR_MAX_DIM)
+    return bsr::report(BSR_EINVAL, "dimension out of range (m=%lld n=%lld k=%lld)", (long long)m, (long long)n,
+                       (long long)k);
+  if (k == 0 || k % KE != 0) return bsr::report(BSR_ESHAPE, "K=%lld must be a positive multiple of 256", (long long)k);
+  if (m == 0 || n == 0) return bsr::report(BSR_OK, "");
+  if (!a || !w_packed || !w_sf_blocked || !out) return bsr::report(BSR_EINVAL, "null pointer");
+  if (!aligned16(a) || !aligned16(w_packed) || !aligned16(w_sf_blocked) || !aligned16(out))
+    return bsr::report(BSR_EALIGN, "a, w_packed, w_sf_blocked and out must be 16-byte aligned");
+  const ProjScratch ps = proj_scratch(m, k);
+  if (!scratch || scratch_bytes < ps.total)
+    return bsr::report(BSR_ESCRATCH, "scratch of %zu bytes needed, %zu given", ps.total,
+                       scratch ? scratch_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(scratch) & 255u) != 0)
+    return bsr::report(BSR_EALIGN, "scratch must be 256-byte aligned");
+  Dev d;
+  int dev = 0;
+  bsr_status st = query_device(d, dev);
+  if (st != BSR_OK) return st;
+  int* status = nullptr;
+  if ((st = bsr::library_status_word(&status)) != BSR_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  uint8_t* a_packed = base + ps.packed;
+  uint8_t* a_e4m3 = base + ps.e4m3;
+  uint8_t* a_sf = base + ps.blocked;
+  float* a_scale2 = reinterpret_cast<float*>(base + ps.scale2);
+  // every tensor map is encoded before the first launch, so a failure
+  // leaves nothing queued
+  GemmLaunch g;
+  if ((st = prepare_gemm(g, a_packed, w_packed, m, n, k, d.num_sms)) != BSR_OK) return st;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = bsr::launch_nvfp4_quant_rows(a, a_packed, a_e4m3, a_scale2, (int)m, (int)k, s, d.num_sms);
+  if (e == cudaSuccess) e = launch_sf_blocked(a_e4m3, a_sf, m, k, s, d.num_sms);
+  if (e == cudaSuccess) e = launch_prepared(g, a_sf, w_sf_blocked, a_scale2, scale2, out, status, m, n, k, s);
+  if (e != cudaSuccess) return bsr::report(BSR_ECUDA, "w4a4 projection launch: %s", cudaGetErrorString(e));
   return bsr::report(BSR_OK, "");
 }
 

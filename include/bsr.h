@@ -138,6 +138,12 @@ bsr_status bsr_gemm(const int8_t* a_i8, const float* a_scale_t, const int8_t* w_
  */
 size_t bsr_proj_scratch_bytes(int64_t m, int64_t k);
 
+/* Activation rows per tile (128, 192 or 256) that the tensor-core GEMM uses
+ * for an M x N problem on the current device: 128 when M <= 128, else the
+ * width whose whole waves of persistent tiles take the least estimated time.
+ * Informational (no launch); 0 if there is no usable device or M, N < 1. */
+int bsr_gemm_block_m(int64_t m, int64_t n);
+
 /*
  * bsr_proj -- gemm_dense_int8.rs, `int8_gemm_faith2_prefill`:
  * out[M, N] = A[M, K] . W[N, K]^T from BF16 A and the requantised weight.
@@ -281,6 +287,30 @@ bsr_status bsr_nvfp4_sf_blocked(const uint8_t* e4m3, uint8_t* blocked, int64_t r
 bsr_status bsr_w4a4_gemm(const uint8_t* a_packed, const uint8_t* a_sf_blocked, const float* a_scale2,
                          const uint8_t* w_packed, const uint8_t* w_sf_blocked, float scale2, uint16_t* out, int64_t m,
                          int64_t n, int64_t k, int* status_dev, void* stream);
+
+/* Scratch bytes bsr_w4a4_proj needs for M activation rows: the quantised
+ * rows (M*K/2 packed bytes, M*K/16 E4M3 bytes), their blocked scales and the
+ * M row scales, each rounded up to 256 bytes (0 for invalid sizes; K % 256
+ * == 0). */
+size_t bsr_w4a4_proj_scratch_bytes(int64_t m, int64_t k);
+
+/*
+ * bsr_w4a4_proj -- the whole W4A4 projection on the tensor cores
+ * (w4a4_proj/fixed.rs, `nvfp4_proj_mx`: quantise the BF16 rows, then the
+ * FP4 product): a [M, K] BF16 -> bsr_nvfp4_quant_rows into scratch ->
+ * bsr_nvfp4_sf_blocked of the row scales -> bsr_w4a4_gemm against w_packed
+ * [N, K/2] with its scales already in the blocked layout (w_sf_blocked, from
+ * bsr_nvfp4_sf_blocked once per weight) and scale2 (host value); out [M, N]
+ * BF16.  Bit-identical to the three calls made separately.  Scratch
+ * (caller-owned, device, 256-byte aligned) of at least
+ * bsr_w4a4_proj_scratch_bytes(M, K); a, w_packed, w_sf_blocked and out
+ * 16-byte aligned; K % 256 == 0.  Timed-out waits are reported through
+ * bsr_device_status().  Every tensor map is encoded before the first
+ * launch: on a non-OK status nothing was queued.
+ */
+bsr_status bsr_w4a4_proj(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_sf_blocked, float scale2,
+                         uint16_t* out, int64_t m, int64_t n, int64_t k, void* scratch, size_t scratch_bytes,
+                         void* stream);
 
 /*
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,

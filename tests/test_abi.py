@@ -161,6 +161,28 @@ def test_w4a4_gemm_argument_errors(L):
     assert L.bsr_w4a4_gemm(None, None, None, None, None, f, None, 0, 8, 256, None, None) == 0
 
 
+def test_w4a4_proj_argument_errors(L):
+    f = ctypes.c_float(1.0)
+    m, k = 64, 512
+    need = L.bsr_w4a4_proj_scratch_bytes(m, k)
+    # packed codes, E4M3 bytes, blocked scales, row scales, each 256-aligned
+    assert need == 16384 + 2048 + 4096 + 256
+    assert L.bsr_w4a4_proj_scratch_bytes(m, 320) == 0 and L.bsr_w4a4_proj_scratch_bytes(0, k) == 0
+    a4 = [_fake(256)] * 3
+    assert L.bsr_w4a4_proj(*a4, f, _fake(256), m, 8, 320, _fake(256), need, None) == 3
+    assert L.bsr_w4a4_proj(*a4, f, _fake(256), m, 8, k, None, 0, None) == 4
+    assert L.bsr_w4a4_proj(*a4, f, _fake(256), m, 8, k, _fake(256), need - 1, None) == 4
+    assert L.bsr_w4a4_proj(*a4, f, _fake(256), m, 8, k, _fake(272), need, None) == 2
+    assert L.bsr_w4a4_proj(*a4, f, _fake(264), m, 8, k, _fake(256), need, None) == 2
+    assert L.bsr_w4a4_proj(None, *a4[:2], f, _fake(256), m, 8, k, _fake(256), need, None) == 1
+    assert L.bsr_w4a4_proj(None, None, None, f, None, 0, 8, k, None, 0, None) == 0
+
+
+def test_gemm_block_m_needs_a_device(L):
+    # informational query: 0 for invalid sizes, and without a usable device
+    assert L.bsr_gemm_block_m(0, 8) == 0 and L.bsr_gemm_block_m(8, -1) == 0
+
+
 def test_scratch_errors(L):
     m, k = 64, 256
     need = L.bsr_proj_scratch_bytes(m, k)

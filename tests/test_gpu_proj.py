@@ -8,8 +8,12 @@
 * the invariants: row bits independent of M and of the other rows (within a
   path), stacked-segment bits, zero inputs -> +0 bits, weight-row permutation,
 * edge shapes (M = 1..129, ragged N, one K stage), the fallback epilogue for
-  scales outside the fast window, and every workload at full size on sampled
-  output rows.
+  scales outside the fast window, and every workload at full size on 64
+  sampled output rows (first and last rows, the ragged tail, the all-zero row,
+  a row with near-zero groups),
+* every activation-tile width the GEMM can choose (128, 192, 256 rows):
+  partials bit-exact and outputs within tolerance on a ragged shape that
+  selects it.
 """
 import numpy as np
 import pytest
@@ -56,6 +60,43 @@ def test_gemm_partials_bit_exact(shape):
     assert_close_bf16(bf16_bits(out), ref, "gemm output")
     # the dump variant and the plain kernel give the same output bits
     assert np.array_equal(bf16_bits(bsr.gemm(a_i8, a_st, w_i8, w_s)), bf16_bits(out))
+
+
+def _shape_for_width(width):
+    """A ragged (M, N) for which the GEMM chooses activation tiles of `width`
+    rows on this device."""
+    for m in (129, 200, 300, 385, 520, 700, 1000, 1300, 2000):
+        for n in (136, 300, 1000, 4000, 9000, 19000):
+            if bsr.gemm_block_m(m, n) == width:
+                return m, n
+    return None
+
+
+@pytest.mark.parametrize("width", [128, 192, 256])
+def test_gemm_partials_each_tile_width(width):
+    shape = _shape_for_width(width)
+    if shape is None:
+        pytest.skip(f"no searched shape selects {width}-row tiles on this device")
+    m, n = shape
+    k = 256
+    w, a = _case(m, n, k, seed=width, recipe="laplace_zero_row", outlier_rows=0.01)
+    w_i8, w_s = _weights(w)
+    a_i8, a_st = bsr.requant_a(up_bf16(a))
+    out, p = bsr.gemm_partials(a_i8, a_st, w_i8, w_s)
+    qa, sa = oracle.requant_a(a)
+    qw, sw = _oracle_w(w, k)
+    ref_p = oracle.block_partials(qa, qw)
+    assert np.array_equal(p.cpu().numpy().astype(np.int64), ref_p)
+    ref = oracle.bf16_rne(oracle.accumulate(ref_p, sa, sw))
+    assert_close_bf16(bf16_bits(out), ref, f"gemm output, {width}-row tiles")
+    assert np.array_equal(bf16_bits(bsr.gemm(a_i8, a_st, w_i8, w_s)), bf16_bits(out))
+    assert bsr.device_status() == 0
+
+
+def test_tile_width_choice_is_valid():
+    for m, n in [(17, 4096), (128, 100), (129, 4096), (2048, 14336), (8192, 4096), (4095, 8192)]:
+        assert bsr.gemm_block_m(m, n) in (128, 192, 256)
+    assert bsr.gemm_block_m(100, 4096) == 128
 
 
 def test_gemm_partials_tiny_workload_in_full(tiny):
@@ -240,15 +281,18 @@ def test_full_size_sampled_rows(name):
     a = up_bf16(d["a_bits"])
     out = bsr.proj(a, w_i8, w_s)
     torch.cuda.synchronize()
-    must = [d["act_info"]["zero_row"]] if "zero_row" in d["act_info"] else []
-    rows = synth.sample_rows(wl.m, 12 if wl.m > 1 else 1, wl.seed, must=must)
+    info = d["act_info"]
+    must = [info["zero_row"]] if "zero_row" in info else []
+    if "near_zero_groups" in info:
+        must.append(int(info["near_zero_groups"][0]) // (wl.k // 32))
+    rows = synth.sample_rows(wl.m, 64 if wl.m > 1 else 1, wl.seed, must=must)
     # oracle weight requantisation on the full weight, then the sampled rows
     qw, sw = _oracle_w(d, wl.k)
     ref = oracle.proj_rows(d["a_bits"][rows], qw, sw)
     got = bf16_bits(out)[rows]
     assert_close_bf16(got, ref, name)
-    if must:
-        zr = int(np.where(rows == must[0])[0][0])
+    if "zero_row" in info:
+        zr = int(np.where(rows == info["zero_row"])[0][0])
         assert np.all(got[zr] == 0)
 
 

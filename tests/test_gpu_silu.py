@@ -50,9 +50,9 @@ def _near_boundary(x, ref_bits, rel=2.0 ** -20):
     return np.abs(np.abs(x) - boundary) <= rel * np.abs(x)
 
 
-def _check_product_bits(g_bits, u_bits, got):
+def _check_product_bits(g_bits, u_bits, got, max_frac=1e-3):
     """Kernel product bits `got` against the exact product; returns the
-    oracle's bits."""
+    oracle's bits.  At most max_frac of the products may differ."""
     ref = oracle.silu_mul_bf16(g_bits, u_bits)
     diff = got != ref
     if np.any(diff):
@@ -64,17 +64,17 @@ def _check_product_bits(g_bits, u_bits, got):
         one_step = np.abs((got[rest] & 0x7FFF).astype(np.int32) - (ref[rest] & 0x7FFF).astype(np.int32)) == 1
         assert np.all(same_sign & one_step), "a product differs by more than one BF16 step"
         assert np.all(_near_boundary(x[rest], ref[rest])), "a product differs away from a rounding boundary"
-        assert rest.sum() <= max(1, 1e-3 * got.size), f"{int(rest.sum())} of {got.size} products differ"
+        assert rest.sum() <= max(1, max_frac * got.size), f"{int(rest.sum())} of {got.size} products differ"
     return ref
 
 
-def _check_quant_arrays(g_bits, u_bits, x_gpu, q_gpu, s_gpu):
+def _check_quant_arrays(g_bits, u_bits, x_gpu, q_gpu, s_gpu, max_frac=1e-3):
     """Codes q_gpu [m, K] and scales s_gpu [m, K/32] of the fused quantiser,
     given the kernel's product bits x_gpu: bit-exact against requant_a of
     that product, and against the oracle's quantiser wherever a group's 32
     products agree with the exact product.  Returns the agreeing fraction."""
     m, k = g_bits.shape
-    ref = _check_product_bits(g_bits, u_bits, x_gpu)
+    ref = _check_product_bits(g_bits, u_bits, x_gpu, max_frac)
     q, s = oracle.requant_a(x_gpu)
     assert np.array_equal(q_gpu, q)
     assert np.array_equal(s_gpu.view(np.uint32), s.view(np.uint32))
@@ -85,12 +85,13 @@ def _check_quant_arrays(g_bits, u_bits, x_gpu, q_gpu, s_gpu):
     return float(agree.mean())
 
 
-def _check_quant(g_bits, u_bits):
+def _check_quant(g_bits, u_bits, max_frac=1e-3):
     m, k = g_bits.shape
     gd, ud = up_bf16(g_bits), up_bf16(u_bits)
     x_gpu = bf16_bits(bsr.silu_mul(gd, ud))
     a_i8, a_st = bsr.requant_silu_a(gd, ud)
-    assert _check_quant_arrays(g_bits, u_bits, x_gpu, a_i8.cpu().numpy(), f32(a_st)[:, :m].T.copy()) > 0.9
+    agree = _check_quant_arrays(g_bits, u_bits, x_gpu, a_i8.cpu().numpy(), f32(a_st)[:, :m].T.copy(), max_frac)
+    assert agree > 0.9
 
 
 @pytest.mark.parametrize("m,k", [(1, 32), (7, 96), (33, 256), (130, 512), (512, 4096)])
@@ -111,7 +112,11 @@ def test_product_over_the_whole_exp_range():
     g[2, :32] = np.linspace(-100, 100, 32)
     u = rng.standard_normal((m, k)) * 10.0 ** rng.uniform(-3, 3, size=(m, k))
     g_bits, u_bits = _bf16(g), _bf16(u)
-    _check_quant(g_bits, u_bits)
+    # Here many products sit exactly on a BF16 midpoint: for 16.6 < g < 36.7
+    # the kernel's 1 + e^-g rounds to 1 in float32, so its product is the
+    # exact g * u of two BF16 values, often a tie, while the exact product
+    # lies just below it.  Those are boundary cases too; allow 0.5%.
+    _check_quant(g_bits, u_bits, max_frac=5e-3)
 
 
 def test_quantiser_near_zero_and_zero_groups():
