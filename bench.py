@@ -46,7 +46,9 @@ if ROOT not in sys.path:
 
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}
-INT8_PER_BF16 = 2.0  # nominal dense int8 / bf16 tensor ratio on B200 (4.5 / 2.25 PFLOP/s)
+INT8_NOMINAL_TOPS = 4500.0  # B200 dense int8 tensor figure (datasheet), for context beside the measured peak
+FP4_PER_BF16 = 4.0  # nominal dense FP4 / bf16 tensor ratio on B200 (9 / 2.25 PFLOP/s)
+ORACLE_MAX_WORKERS = 16  # host processes of the all-cores oracle baseline
 # The exact per-block rescale costs 2 FP32 FMAs per output element and 32-wide
 # K block (= 64 int8 ops); the FP32 pipe retires 128 FMAs per clock per SM.
 OPS_PER_SM_CLOCK_FMA_BOUND = 64 * 128 / 2
@@ -208,6 +210,48 @@ class ClockSampler:
         }
 
 
+def measure_int8_peak(device, n=8192, reps=10):
+    """Dense int8 tensor throughput of this GPU in TOPS: torch._int_mm (cuBLAS
+    int8 GEMM, int32 out) of n x n x n, best of `reps` launches timed with
+    CUDA events on the current stream."""
+    import torch
+
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=device).t()  # column-major operand
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    torch.cuda.empty_cache()
+    return 2.0 * n ** 3 / (best / 1e3) / 1e12
+
+
+def host_cpu():
+    """CPU model and logical core count of the host running the oracle."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count() or 1
+    return {"model": model, "nproc": usable}
+
+
 def roofline(bound, achieved, peak, unit, traffic):
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": (achieved / peak) if peak else None, "traffic": traffic}
@@ -216,7 +260,8 @@ def roofline(bound, achieved, peak, unit, traffic):
 # translation unit of each measured kernel; with the csrc headers it includes
 # and the C-ABI layer that picks its launch parameters, these are the sources
 # its DRAM traffic depends on
-KERNEL_UNITS = {"decode_kernel": "decode.cu", "gemm_kernel": "gemm_tc.cu"}
+KERNEL_UNITS = {"decode_kernel": "decode.cu", "gemm_kernel": "gemm_tc.cu", "requant_a_kernel": "requant.cu",
+                "requant_w_kernel": "requant.cu", "requant_silu_a_kernel": "silu.cu"}
 LAUNCH_LAYER = "api.cu"
 
 
@@ -280,11 +325,14 @@ def stored_traffic(kernel: str, workload: str):
 # ---------------------------------------------------------------------------
 
 
-def workload_desc(wl):
+def workload_desc(wl, world=1):
+    """The `config` object of the bench line: the same for both arms."""
     m, n, k = wl.shape
+    l2 = ("rotating copies of the requantised weight covering >= 3x L2 across the K steps of one CUDA-graph replay"
+          if m <= 16 else "flushed before every timed step (256 MiB device write, outside the step events)")
     return {"workload": f"{wl.name}: M={m} N={n} K={k} (NVFP4 weight, BF16 activations '{wl.act}')",
-            "m": m, "n": n, "k": k, "seed": wl.seed,
-            "l2": "flushed before every timed step (256 MiB device write, outside the step events)"}
+            "m": m, "n": n, "k": k, "seed": wl.seed, "l2": l2,
+            "parallelism": f"replicas x{world} (no exchange step)"}
 
 
 def input_hashes(d):
@@ -483,6 +531,23 @@ class Gpu:
 # ---------------------------------------------------------------------------
 
 
+_POOL_W = None
+
+
+def _pool_init(w_i8, w_s):
+    """Worker start-up of the all-cores oracle: keep the requantised weight."""
+    global _POOL_W
+    _POOL_W = (w_i8, w_s)
+
+
+def _pool_rows(a_rows):
+    """One oracle projection of the given activation rows (in a worker)."""
+    import oracle
+
+    oracle.proj_rows(a_rows, *_POOL_W)
+    return len(a_rows)
+
+
 class OracleRunner:
     """Times the CPU oracle on a bounded sample of a workload.  The weight
     requantisation runs once, outside the timing (as on the GPU)."""
@@ -507,12 +572,32 @@ class OracleRunner:
         return time.perf_counter() - t0
 
     def per_row_seconds(self, budget_s):
-        """Mean oracle seconds per activation row over a sample bounded by budget_s."""
+        """Mean oracle seconds per activation row on one core, over a sample
+        bounded by budget_s."""
         done, spent = 0, 0.0
         while spent < budget_s and done < 1000:
             spent += self.sample_step(1)
             done += 1
         return spent / done, done
+
+    def per_row_seconds_all_cores(self, single_row_s, budget_s):
+        """Wall seconds per activation row with the sampled rows spread over
+        host worker processes (spawned, one per core up to
+        ORACLE_MAX_WORKERS): the oracle unchanged, run side by side.
+        Returns (seconds per row, rows, workers)."""
+        import multiprocessing
+
+        workers = max(1, min(host_cpu()["nproc"], ORACLE_MAX_WORKERS))
+        per_worker = max(1, int(budget_s / max(single_row_s, 1e-6)))
+        nrows = workers * per_worker
+        tasks = [self.a[self.rows[i % len(self.rows)]][None] for i in range(nrows)]
+        ctx = multiprocessing.get_context("spawn")
+        with ctx.Pool(workers, initializer=_pool_init, initargs=(self.w_i8, self.w_s)) as pool:
+            pool.map(_pool_rows, tasks[:workers], chunksize=1)  # warm-up: every worker once
+            t0 = time.perf_counter()
+            pool.map(_pool_rows, tasks, chunksize=per_worker)
+            wall = time.perf_counter() - t0
+        return wall / nrows, nrows, workers
 
 
 def units_per_step(wl):
@@ -522,18 +607,37 @@ def units_per_step(wl):
     return prefill_ops(m, n, k) / 1e12, "TOPS", "int8 block-scaled proj TOPS (prefill, incl. requant)"
 
 
-def cpu_baseline(name, budget_s):
+def cpu_baseline(name, budget_s, all_cores=True):
+    """The oracle as it stands on the host: one core, and the same rows
+    spread over worker processes on all cores (up to ORACLE_MAX_WORKERS).
+    Step time = time per activation row x M (extrapolated when M > 1)."""
     r = OracleRunner(name)
     per_row, rows = r.per_row_seconds(budget_s)
     units, unit, _ = units_per_step(r.wl)
-    step_s = per_row * r.wl.m
-    sample = (f"{rows} oracle projection(s) of one activation row each against the full requantised weight, "
-              f"timed on the host; step time = per-row time x M={r.wl.m}" + (" (extrapolated)" if r.wl.m > 1 else ""))
-    return {"value": units / step_s, "unit": unit, "cores": 1, "kind": "oracle", "sample": sample,
-            "ms_per_step": step_s * 1e3}
+    m = r.wl.m
+    ext = " (extrapolated)" if m > 1 else ""
+    host = host_cpu()
+    res = {"value": units / (per_row * m), "unit": unit, "cores": 1, "kind": "oracle",
+           "sample": (f"{rows} oracle projection(s) of one sampled activation row each against the full requantised "
+                      f"weight on one core; step time = per-row time x M={m}{ext}"),
+           "ms_per_step": per_row * m * 1e3, "cpu_model": host["model"], "nproc": host["nproc"]}
+    if all_cores:
+        per_row_p, prow, workers = r.per_row_seconds_all_cores(per_row, budget_s / 2)
+        res["all_cores"] = {"value": units / (per_row_p * m), "unit": unit, "cores": workers,
+                            "ms_per_step": per_row_p * m * 1e3,
+                            "sample": (f"{prow} sampled rows over {workers} spawned worker processes (wall time); "
+                                       f"step time = wall time per row x M={m}{ext}")}
+    return res
 
 
 def reference_main(args):
+    """The reference arm: the CPU oracle as it stands, on the host cores, on
+    the GPU arm's workload, metric and unit.  Each step projects one sampled
+    activation row per worker process (spawned, one per core up to
+    ORACLE_MAX_WORKERS) against the full requantised weight; step time = wall
+    time per row x M."""
+    import multiprocessing
+
     rank, world, _ = dist_env()
     if rank != 0:
         return 0
@@ -542,18 +646,29 @@ def reference_main(args):
     wl = synth.WORKLOADS[args.workload]
     r = OracleRunner(args.workload)
     units, unit, metric = units_per_step(wl)
-    for _ in range(args.warmup):
-        r.sample_step(1)
-    t = [r.sample_step(1) for _ in range(args.steps)]
+    host = host_cpu()
+    workers = max(1, min(host["nproc"], ORACLE_MAX_WORKERS))
+    rows = [r.a[r.rows[i % len(r.rows)]][None] for i in range(workers)]
+    ctx = multiprocessing.get_context("spawn")
+    with ctx.Pool(workers, initializer=_pool_init, initargs=(r.w_i8, r.w_s)) as pool:
+        for _ in range(args.warmup):
+            pool.map(_pool_rows, rows, chunksize=1)
+        t = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            pool.map(_pool_rows, rows, chunksize=1)
+            t.append((time.perf_counter() - t0) / workers)
     step_s = float(np.mean(t)) * wl.m
     value = units / step_s
+    sample = (f"each step: {workers} sampled activation rows, one per worker process, against the full requantised "
+              f"weight; step time = wall time per row x M={wl.m}" + (" (extrapolated)" if wl.m > 1 else ""))
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded generator)", "impl": "reference",
-            "config": {**workload_desc(wl), "inputs_sha256": r.hashes},
-            "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
-                             "sample": f"each step: the oracle on 1 of {len(r.rows)} sampled activation rows against the "
-                                       f"full requantised weight; step time = per-row time x M={wl.m}"},
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic (seeded generator; no dataset or trained weights)",
+            "impl": "reference",
+            "config": {**workload_desc(wl, args.gpus), "inputs_sha256": r.hashes},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": workers, "kind": "oracle", "sample": sample,
+                             "cpu_model": host["model"], "nproc": host["nproc"]},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -568,27 +683,50 @@ def mean_ms(times):
     return float(np.mean(times))
 
 
-def prefill_extra(name, device, steps, warmup, peaks, cpu=True):
-    """Secondary measurement of one prefill workload (rank-local)."""
+def prefill_extra(name, device, steps, warmup, peaks, int8_peak, pci, cpu=True, cpu_budget=6.0):
+    """Full measurement record of one prefill workload (rank-local): the step
+    (requant_a + GEMM), the GEMM alone with its roofline, the two
+    requantisations, clocks sampled during the GEMM timing, the end-to-end
+    step through the public API, and the oracle baseline."""
     g = Gpu(name, device)
     m, n, k = g.wl.shape
     ops = prefill_ops(m, n, k)
     t_step = mean_ms(g.timed(g.step, steps, warmup))
-    t_gemm = mean_ms(g.timed_gemm_only(steps, warmup))
+    with ClockSampler(pci) as clk:
+        t_gemm = mean_ms(g.timed_gemm_only(steps, warmup))
     t_ra = mean_ms(g.timed_requant_a_only(steps, warmup))
     t_rw = mean_ms(g.timed_requant_w_only(steps, warmup))
+    t_e2e = mean_ms(g.timed(g.step_e2e, max(3, steps // 2), 1))
     g.check_status()
-    int8_peak = peaks["bf16_tflops"] * INT8_PER_BF16
-    fma_peak = fma_bound_tops(g.num_sms, peaks["sm_max_mhz"])
+    clocks = clk.summary()
+    mhz = clocks["sm_mhz"] or peaks["sm_max_mhz"]
+    fma_peak = fma_bound_tops(g.num_sms, mhz)
+    achieved = ops / t_gemm / 1e9
+    rl = roofline("alu", achieved, fma_peak, "TOPS", stored_traffic("gemm_kernel", name))
+    rl.update({
+        "kernel": "gemm_kernel", "tile_m": g.bsr.gemm_block_m(m, n),
+        "peak_source": (f"2 FP32 FMAs per element and 32-block at 128 FMA/clk/SM x {g.num_sms} SMs x {mhz:g} MHz "
+                        f"(median SM clock sampled during the GEMM timing)"),
+        "tensor_peak": int8_peak, "tensor_frac": achieved / int8_peak,
+        "tensor_peak_source": "torch._int_mm int8 8192^3, best of 10, measured in this run",
+        "tensor_peak_nominal": INT8_NOMINAL_TOPS, "tensor_frac_nominal": achieved / INT8_NOMINAL_TOPS,
+    })
+    ra_gbs = m * k * 3.125 / t_ra / 1e6
+    rw_gbs = n * k * 1.6875 / t_rw / 1e6
     res = {
         "shape": [m, n, k],
         "tops_incl_requant": ops / t_step / 1e9,
-        "gemm_tops": ops / t_gemm / 1e9,
-        "gemm_frac_of_int8_peak": ops / t_gemm / 1e9 / int8_peak,
-        "gemm_frac_of_fma_bound": ops / t_gemm / 1e9 / fma_peak,
-        "requant_a_gbs": m * k * 3.125 / t_ra / 1e6,
-        "requant_w_gbs": n * k * 1.6875 / t_rw / 1e6,
-        "ms": {"step": t_step, "gemm": t_gemm, "requant_a": t_ra, "requant_w": t_rw},
+        "ms_step": t_step,
+        "roofline": rl,
+        "requant_a": {"gbs": ra_gbs, "frac_of_hbm": ra_gbs / peaks["hbm_gbs"], "ms": t_ra,
+                      "bytes": m * k * 3.125, "traffic": stored_traffic("requant_a_kernel", name)},
+        "requant_w": {"gbs": rw_gbs, "frac_of_hbm": rw_gbs / peaks["hbm_gbs"], "ms": t_rw,
+                      "bytes": n * k * 1.6875, "traffic": stored_traffic("requant_w_kernel", name)},
+        "clocks": clocks,
+        "e2e": {"value": ops / t_e2e / 1e9, "unit": "TOPS", "h2d_bytes_per_step": 2 * m * k,
+                "d2h_bytes_per_step": 2 * m * n, "ms_per_step": t_e2e,
+                "how": "eager calls per step (activations copied in from pinned host memory, projection, output "
+                       "copied back to pinned host memory)"},
     }
     if g.wl.act == "silu_mul":
         res["silu"] = silu_extra(g, steps, warmup, cpu)
@@ -596,7 +734,62 @@ def prefill_extra(name, device, steps, warmup, peaks, cpu=True):
     import torch
 
     torch.cuda.empty_cache()
+    if cpu:
+        res["cpu_baseline"] = cpu_baseline(name, cpu_budget)
     return res
+
+
+def w4a4_gemm_extra(device, steps, warmup, peaks):
+    """The W4A4 projection on the tensor cores (block-scaled FP4 MMA) on the
+    2048 x 14336 x 4096 shape with the FFN-up inputs: the composite entry
+    (row quantiser, scale relayout, GEMM) and the GEMM alone, against the FP4
+    tensor figure (measured bf16 peak x the nominal FP4/bf16 ratio)."""
+    import torch
+
+    import block_scaled_precision_requant_b200 as bsr
+    from block_scaled_precision_requant_b200 import synth
+
+    d = synth.make_workload("ffn_up")
+    m, n, k = d["workload"].shape
+    wp = torch.from_numpy(d["w_packed"]).to(device)
+    w_sf = bsr.sf_blocked(torch.from_numpy(d["w_e4m3"]).to(device))
+    a = torch.from_numpy(d["a_bits"].view(np.int16)).view(torch.bfloat16).to(device)
+    s2 = float(d["scale2"])
+    out = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+    scratch = torch.empty((bsr.w4a4_proj_scratch_bytes(m, k),), dtype=torch.uint8, device=device)
+    ap, ae, as2 = bsr.quant_nvfp4_rows(a)
+    a_sf = bsr.sf_blocked(ae)
+    status = torch.zeros((1,), dtype=torch.int32, device=device)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.mean(ts))
+
+    t_proj = timed(lambda: bsr.w4a4_proj(a, wp, w_sf, s2, out, scratch))
+    t_gemm = timed(lambda: bsr.w4a4_gemm(ap, a_sf, as2, wp, w_sf, s2, out, status))
+    if int(status.item()) != 0 or bsr.device_status() != 0:
+        raise RuntimeError("W4A4 GEMM: a pipeline wait timed out")
+    ops = prefill_ops(m, n, k)
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    del wp, w_sf, a, out, scratch, ap, ae, as2, a_sf, flush
+    torch.cuda.empty_cache()
+    return {"shape": [m, n, k], "tops_proj": ops / t_proj / 1e9, "ms_proj": t_proj,
+            "gemm_tops": ops / t_gemm / 1e9, "ms_gemm": t_gemm,
+            "fp4_peak": fp4_peak, "gemm_frac_of_fp4_peak": ops / t_gemm / 1e9 / fp4_peak,
+            "peak_source": f"measured bf16 burst x {FP4_PER_BF16:g} (nominal dense FP4/bf16 ratio)",
+            "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
 
 
 def stacked_decode_extra(device, steps, peaks, cpu=True):
@@ -872,6 +1065,8 @@ def gpu_main(args):
     props = torch.cuda.get_device_properties(dev)
     pci = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
     peaks, peak_src = load_peaks()
+    extras = not args.no_extra and world == 1
+    int8_peak = measure_int8_peak(dev) if extras or args.workload != "decode" else None
 
     g = Gpu(args.workload, dev)
     wl = g.wl
@@ -891,13 +1086,14 @@ def gpu_main(args):
     if decode:
         t_kernel = t_steps  # the step is one launch of the decode kernel
         kernel = "decode_kernel"
+        t_single = g.timed(lambda: g.bsr.decode(g.a, g.w_i8, g.w_s, g.out), args.steps, args.warmup)
     else:
-        t_kernel = g.timed_gemm_only(args.steps, args.warmup)
+        with ClockSampler(pci) as clk_kernel:
+            t_kernel = g.timed_gemm_only(args.steps, args.warmup)
         kernel = "gemm_kernel"
     t_rw = g.timed_requant_w_only(min(args.steps, 20), args.warmup)
     g.check_status()
-    w4 = (w4a16_extra(g, max(args.steps, 20), peaks, cpu=not args.no_cpu)
-          if decode and not args.no_extra and world == 1 else None)
+    w4 = w4a16_extra(g, max(args.steps, 20), peaks, cpu=not args.no_cpu) if decode and extras else None
 
     ms_step, ms_e2e, ms_kernel, ms_rw, ms_e2e_eager = dist_max(
         [mean_ms(t_steps), mean_ms(t_e2e), mean_ms(t_kernel), mean_ms(t_rw), mean_ms(t_e2e_eager)],
@@ -907,29 +1103,31 @@ def gpu_main(args):
     if decode:
         rl = roofline("hbm", decode_bytes(m, n, k) / (ms_kernel / 1e3) / 1e9, peaks["hbm_gbs"], "GB/s",
                       stored_traffic(kernel, wl.name))
+        rl["peak_source"] = f"{peak_src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
+        rl["single_launch"] = {"ms": mean_ms(t_single),
+                               "gbs": decode_bytes(m, n, k) / (mean_ms(t_single) / 1e3) / 1e9,
+                               "how": "one eager launch per step, L2 flushed before each (no overlap of steps)"}
     else:
         # the GEMM is bound by the FP32 pipe (the exact rescale), not by the
-        # tensor pipe: report against that bound, and the tensor peak beside it
+        # tensor pipe: report against that bound at the sampled clock, and the
+        # measured int8 tensor peak beside it
         achieved = prefill_ops(m, n, k) / (ms_kernel / 1e3) / 1e12
-        rl = roofline("alu", achieved, fma_bound_tops(props.multi_processor_count, peaks["sm_max_mhz"]), "TOPS",
+        mhz = clk_kernel.summary()["sm_mhz"] or peaks["sm_max_mhz"]
+        rl = roofline("alu", achieved, fma_bound_tops(props.multi_processor_count, mhz), "TOPS",
                       stored_traffic(kernel, wl.name))
-        rl["tensor_peak"] = peaks["bf16_tflops"] * INT8_PER_BF16
-        rl["tensor_frac"] = achieved / rl["tensor_peak"]
+        rl["tensor_peak"] = int8_peak
+        rl["tensor_frac"] = achieved / int8_peak
+        rl["tensor_peak_nominal"] = INT8_NOMINAL_TOPS
+        rl["peak_source"] = (f"2 FP32 FMAs per element and 32-block at 128 FMA/clk/SM x {props.multi_processor_count} "
+                             f"SMs x {mhz:g} MHz (median SM clock sampled during the GEMM timing); tensor_peak: "
+                             f"torch._int_mm int8 8192^3 measured in this run")
     rl["kernel"] = kernel
-    rl["peak_source"] = (f"{peak_src} (HBM copy)" if decode else
-                         f"2 FP32 FMAs per element and 32-block at 128 FMA/clk/SM x {props.multi_processor_count} SMs "
-                         f"x {peaks['sm_max_mhz']:g} MHz; tensor_peak: {peak_src} bf16 cuBLAS burst x "
-                         f"{INT8_PER_BF16:g} (nominal int8/bf16 ratio)")
 
     line = {
         "metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8",
         "data": "synthetic (seeded generator; no dataset or trained weights)",
-        "config": {**workload_desc(wl), "parallelism": f"replicas x{world} (no exchange step)",
-                   "inputs_sha256": input_hashes(g.host),
-                   **({"l2": f"{getattr(g, 'rotating_copies', 0)} rotating copies of the requantised weight "
-                             f"(>= 3x L2) across the K steps of one CUDA-graph replay; e2e flushes L2 per step"}
-                      if decode else {})},
+        "config": {**workload_desc(wl, world), "inputs_sha256": input_hashes(g.host)},
         "roofline": rl,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": 2 * m * k, "d2h_bytes_per_step": 2 * m * n,
                 "how": ("CUDA graph of the K steps (copy in, projection, copy out each step)" if decode else
@@ -938,22 +1136,40 @@ def gpu_main(args):
                 "ms_per_step": ms_e2e},
         "gpu_launches": g.launches_per_step() * args.steps,
         "clocks": clk.summary(),
+        "int8_peak_tops": int8_peak,
         "requant_w": {"gbs": n * k * 1.6875 / (ms_rw / 1e3) / 1e9, "ms": ms_rw,
                       "frac_of_hbm": n * k * 1.6875 / (ms_rw / 1e3) / 1e9 / peaks["hbm_gbs"]},
     }
+    if decode:
+        line["l2_rotating_copies"] = getattr(g, "rotating_copies", None)
     host = g.host
     del g
     torch.cuda.empty_cache()
-    if not args.no_extra and world == 1:
-        extra = {}
+    if extras:
+        detail = {}
         for name in ("ffn_up", "ffn_down", "square_ragged"):
             if name != args.workload:
-                extra[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks,
-                                            cpu=not args.no_cpu)
-        line["prefill"] = extra
+                detail[name] = prefill_extra(name, dev, min(args.steps, 10), min(args.warmup, 3) or 1, peaks,
+                                             int8_peak, pci, cpu=not args.no_cpu)
+        # flat summary (scalars only) beside the per-workload records
+        flat = {}
+        for name, r in detail.items():
+            flat[f"{name}_tops_incl_requant"] = r["tops_incl_requant"]
+            flat[f"{name}_gemm_tops"] = r["roofline"]["achieved"]
+            flat[f"{name}_gemm_frac_fp32_bound"] = r["roofline"]["frac"]
+            flat[f"{name}_gemm_frac_int8_peak"] = r["roofline"]["tensor_frac"]
+            flat[f"{name}_requant_a_gbs"] = r["requant_a"]["gbs"]
+            flat[f"{name}_sm_mhz"] = r["clocks"]["sm_mhz"]
+            flat[f"{name}_e2e_tops"] = r["e2e"]["value"]
+        line["prefill"] = flat
+        line["prefill_detail"] = detail
         if w4 is not None:
             line["w4a16_decode"] = w4
         line["stacked_prefill"] = stacked_prefill_extra(dev, min(args.steps, 10), 3)
+        try:
+            line["w4a4_gemm"] = w4a4_gemm_extra(dev, min(args.steps, 10), 3, peaks)
+        except Exception as exc:  # noqa: BLE001 - reported in the line
+            line["w4a4_gemm"] = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         if decode:
             line["stacked_decode"] = stacked_decode_extra(dev, max(args.steps, 20), peaks, cpu=not args.no_cpu)
             try:  # the last GPU work of the run: an error here costs only this entry

@@ -77,17 +77,6 @@ constexpr int BN = 128;          // weight rows per tile (MMA M, TMEM lanes)
 constexpr int KBS = 4;           // 32-blocks per stage
 constexpr int KS = 32 * KBS;     // bytes of K per stage (one 128-byte swizzle row)
 constexpr int EPI_WARP0 = 4;
-constexpr int EPI_WARPS = 8;
-constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);  // 384
-// Register split: launched with 384 x 168 = 64512 registers; the control
-// warpgroup (warps 0-3) drops to 56 and the two epilogue warpgroups rise to
-// 224: 128 x 56 + 256 x 224 = 64512.
-constexpr int LAUNCH_REGS = 168;
-constexpr int CTRL_REGS = 56;
-constexpr int EPI_REGS = 224;
-static_assert(THREADS * LAUNCH_REGS <= 65536, "launch register budget");
-static_assert(128 * CTRL_REGS + 32 * EPI_WARPS * EPI_REGS <= THREADS * LAUNCH_REGS,
-              "register split exceeds the launch allocation");
 constexpr uint32_t TMEM_COLS = 512;
 // Constant operand of the bias MMA: 8 KB of 0x80 bytes read through an
 // unswizzled K-major descriptor (core matrices 8 rows x 16 bytes; 128 bytes
@@ -96,6 +85,23 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int CONST_BYTES = 8192;
 constexpr uint32_t kBias = 1u << 19;  // = 32 * 128 * 128
 constexpr size_t kSmemPerCta = 232448;  // 227 KB opt-in limit of sm_100
+
+// Epilogue shape: EW epilogue warps (8 or 12: two or three per scheduler)
+// and CW-column tensor-memory chunks (16 or 32).  Register split: the CTA is
+// launched with THREADS x LAUNCH_REGS registers; the control warpgroup
+// (warps 0-3) drops to CTRL_REGS and the epilogue warpgroups rise to EPI_REGS.
+template <int EW>
+struct Warps {
+  static constexpr int EPI_WARPS = EW;
+  static constexpr int THREADS = 32 * (EPI_WARP0 + EW);
+  static constexpr int LAUNCH_REGS = EW == 8 ? 168 : 128;
+  static constexpr int CTRL_REGS = EW == 8 ? 56 : 32;
+  static constexpr int EPI_REGS = EW == 8 ? 224 : 160;
+  static_assert(EW == 8 || EW == 12, "two or three epilogue warps per scheduler");
+  static_assert(THREADS * LAUNCH_REGS <= 65536, "launch register budget");
+  static_assert(128 * CTRL_REGS + 32 * EW * EPI_REGS <= THREADS * LAUNCH_REGS,
+                "register split exceeds the launch allocation");
+};
 
 template <int BM>
 struct Tile {
@@ -108,15 +114,12 @@ struct Tile {
   static constexpr int OFF_WS = W_TILE + A_TILE;
   static constexpr int OFF_AS = OFF_WS + WS_TILE;
   static constexpr int TBUF = (int)TMEM_COLS / BM;  // tensor-memory ring depth
-  static constexpr int COLS_W = BM / 2;             // columns per epilogue warp
-  static constexpr int CHUNKS = COLS_W / 16;        // 16-column tensor-memory loads
   static constexpr int STAGES_FIT = (int)((kSmemPerCta - 1024 - CONST_BYTES - 512) / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT < 6 ? STAGES_FIT : 6;
   static constexpr uint32_t IDESC = idesc_i8(BN, BM);
   static constexpr uint32_t IDESC_BIAS = IDESC & ~((7u << 7) | (7u << 10));  // u8 x u8
   static_assert(KBS % TBUF == 0, "buffer index pattern");
   static_assert(BM % 32 == 0 && BM <= 256, "MMA N and the scale-prep lanes");
-  static_assert(CHUNKS >= 2, "the epilogue pipelines its tensor-memory loads over >= 2 chunks");
   static_assert(STAGES >= 3, "shared-memory ring");
 };
 
@@ -156,8 +159,12 @@ __device__ __forceinline__ uint64_t smem_desc_const(uint32_t saddr) {
 // Ties 16 registers written by a tensor-memory load to this point of the
 // program: placed after tcgen05.wait::ld, it keeps the compiler from moving
 // their uses above the wait.
-__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[8]) {
-  asm volatile("" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]));
+template <int R>
+__device__ __forceinline__ void regs_after_wait(uint32_t (&r)[R]) {
+#pragma unroll
+  for (int i = 0; i < R; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
+                      "+r"(r[i + 6]), "+r"(r[i + 7]));
 }
 
 // 16 lanes x 128 bits, repeated 4 times along the columns (16 columns):
@@ -169,6 +176,11 @@ __device__ __forceinline__ void tmem_ld_16x128b_x4(uint32_t taddr, uint32_t (&r)
                : "r"(taddr));
 }
 
+// One CW-column chunk of 16 lanes: x4 (16 columns, 8 registers) or x8
+// (32 columns, 16 registers).
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[8]) { tmem_ld_16x128b_x4(taddr, r); }
+__device__ __forceinline__ void tmem_ld_chunk(uint32_t taddr, uint32_t (&r)[16]) { tmem_ld_16x128b_x8(taddr, r); }
+
 // Bounded wait that ignores the abort flag (used while draining).
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer_ns();
@@ -178,16 +190,23 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
-template <int BM, bool DUMP>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int BM, int EW, int CW, bool DUMP>
+__global__ void __launch_bounds__(Warps<EW>::THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_a,
                 const __grid_constant__ CUtensorMap tm_ws, const __grid_constant__ CUtensorMap tm_as,
                 __nv_bfloat16* __restrict__ out, int32_t* __restrict__ partials, int* __restrict__ status, int m,
                 int n, int k, int n_tiles, int m_tiles, int m_fastest, long long ldo) {
   using T = Tile<BM>;
+  using WG = Warps<EW>;
   constexpr int STAGES = T::STAGES;
   constexpr int TBUF = T::TBUF;
-  constexpr int CHUNKS = T::CHUNKS;
+  constexpr int EPI_WARPS = WG::EPI_WARPS;
+  constexpr int HALVES = EW / 4;            // column groups of epilogue warps
+  constexpr int COLS_W = BM / HALVES;       // columns per epilogue warp
+  constexpr int CHUNKS = COLS_W / CW;
+  constexpr int CR = CW / 2;                // registers of one 16-lane chunk load
+  constexpr int KK = CW / 4;                // columns of a chunk per thread
+  static_assert(COLS_W % CW == 0 && CHUNKS >= 2, "the epilogue pipelines its loads over >= 2 chunks");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte-swizzled tiles, keeping the pointer
   // derived from the shared array so accesses stay shared-space loads
@@ -227,7 +246,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_alloc(&ctrl->tmem_base, TMEM_COLS);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < CONST_BYTES / 16; i += THREADS)
+  for (int i = threadIdx.x; i < CONST_BYTES / 16; i += WG::THREADS)
     reinterpret_cast<uint4*>(const_tile)[i] = make_uint4(0x80808080u, 0x80808080u, 0x80808080u, 0x80808080u);
   fence_proxy_async_smem();
   tc_fence_before();
@@ -249,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   };
 
   if (warp < EPI_WARP0) {
-    setmaxnreg_dec<CTRL_REGS>();
+    setmaxnreg_dec<WG::CTRL_REGS>();
     if (warp == 0) {
       // -------------------------------------------------------------- TMA
       if (lane == 0) {
@@ -348,17 +367,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
             for (int kb = 0; kb < KBS; ++kb) wsf[kb * BN + q * 32 + (lane & 7) * 4 + (lane >> 3)] = w4[kb] * fw;
           }
-          // Activation scales [kb][m], m = 16g + 4j + r  ->  [kb][g][r][j]
-          // (g = 16-column group, r = t%4 of the epilogue thread, j = its
-          // column index within the group): a permutation inside each group.
-          // Lane L takes m = 32G + L, i.e. group 2G + L/16, j = (L/4)%4.
+          // Activation scales [kb][m], m = CW*g + 4j + r  ->  [kb][g][r][j]
+          // (g = CW-column chunk, r = t%4 of the epilogue thread, j = its
+          // column index within the chunk): a permutation inside each chunk.
+          // Lane L takes m = 32G + L: chunk offset (L/CW)*CW, j = (L%CW)/4.
 #pragma unroll 1
           for (int kb = 0; kb < KBS; ++kb) {
             float av[BM / 32];
 #pragma unroll
             for (int g = 0; g < BM / 32; ++g) av[g] = asf[kb * BM + g * 32 + lane];
             __syncwarp();
-            const int dst = (lane >> 4) * 16 + (lane & 3) * 4 + ((lane >> 2) & 3);
+            const int dst = (lane / CW) * CW + (lane & 3) * (CW / 4) + (lane % CW) / 4;
 #pragma unroll
             for (int g = 0; g < BM / 32; ++g) asf[kb * BM + g * 32 + dst] = av[g] * fa;
           }
@@ -374,24 +393,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     prep_done:;
     }
   } else {
-    setmaxnreg_inc<EPI_REGS>();
+    setmaxnreg_inc<WG::EPI_REGS>();
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;
     const int h = (warp - EPI_WARP0) >> 2;
     const int l8 = lane >> 2;
     const int c4 = lane & 3;
-    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * T::COLS_W);
+    const uint32_t tl = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * COLS_W);
     const int my_tiles = (num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const uint32_t smem_base = smem_u32(smem);
     const uint32_t ws_off = T::OFF_WS + (uint32_t)(q * 32 + l8 * 4) * 4u;                // + kb*BN*4
-    const uint32_t as_off = T::OFF_AS + (uint32_t)(h * T::COLS_W + c4 * 4) * 4u;         // + kb*BM*4 + c*64
+    const uint32_t as_off = T::OFF_AS + (uint32_t)(h * COLS_W + c4 * KK) * 4u;           // + kb*BM*4 + c*CW*4
 
     // open the tensor-memory ring
 #pragma unroll
     for (int b = 0; b < TBUF; ++b) mbar_arrive_lane0(&ctrl->tempty[b], lane);
 
-    float2 acc[CHUNKS][2][4];  // acc[c][j][k]: rows (l8 + 16j, l8 + 16j + 8), column 16c + c4 + 4k
-    uint32_t ra[2][8], rb[2][8];
+    float2 acc[CHUNKS][2][KK];  // acc[c][j][k]: rows (l8 + 16j, l8 + 16j + 8), column CW*c + c4 + 4k
+    uint32_t ra[2][CR], rb[2][CR];
 
     const int total_st = my_tiles * kstages;
     int tile = blockIdx.x, n0 = 0, m0 = 0, kst = 0;
@@ -399,14 +418,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t st_addr = smem_base;
     uint32_t itg = 0;
 
-    auto dump = [&](int c, int b, const uint32_t (&x)[8], const uint32_t (&y)[8]) {
+    auto dump = [&](int c, int b, const uint32_t (&x)[CR], const uint32_t (&y)[CR]) {
       if constexpr (DUMP) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int nn = n0 + q * 32 + l8 + 8 * i;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int mm = m0 + h * T::COLS_W + c * 16 + c4 + 4 * kk;
+          for (int kk = 0; kk < KK; ++kk) {
+            const int mm = m0 + h * COLS_W + c * CW + c4 + 4 * kk;
             const uint32_t v = (i < 2) ? x[2 * kk + (i & 1)] : y[2 * kk + (i & 1)];
             if (nn < n && mm < m) partials[((size_t)mm * n + nn) * nb + b] = (int)v - (int)kBias;
           }
@@ -433,8 +452,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!mbar_wait(&ctrl->tfull[buf], par, abort_flag, status, DEV_ERR_TIMEOUT_EPI)) return false;
       tc_fence_after();
       const uint32_t tb = tl + buf * BM;
-      tmem_ld_16x128b_x4(tb, ra[0]);
-      tmem_ld_16x128b_x4(tb + (16u << 16), rb[0]);
+      tmem_ld_chunk(tb, ra[0]);
+      tmem_ld_chunk(tb + (16u << 16), rb[0]);
       tc_wait_ld();
       regs_after_wait(ra[0]);
       regs_after_wait(rb[0]);
@@ -444,15 +463,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         // the fast path loads the next chunk while it rescales this one; the
         // exotic path (rare) loads it afterwards and keeps one buffer live
         if (!EXO && c + 1 < CHUNKS) {
-          tmem_ld_16x128b_x4(tb + 16u * (c + 1), ra[cur ^ 1]);
-          tmem_ld_16x128b_x4(tb + 16u * (c + 1) + (16u << 16), rb[cur ^ 1]);
+          tmem_ld_chunk(tb + (uint32_t)CW * (c + 1), ra[cur ^ 1]);
+          tmem_ld_chunk(tb + (uint32_t)CW * (c + 1) + (16u << 16), rb[cur ^ 1]);
         }
-        const float4 A0 = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u) + (uint32_t)c * 64u);
-        const float av[4] = {A0.x, A0.y, A0.z, A0.w};
+        float av[KK];
+#pragma unroll
+        for (int v = 0; v < KK / 4; ++v) {
+          const float4 A = lds_f32x4(st_addr + as_off + (uint32_t)kb * (BM * 4u) + (uint32_t)c * (CW * 4u) + 16u * v);
+          av[4 * v] = A.x;
+          av[4 * v + 1] = A.y;
+          av[4 * v + 2] = A.z;
+          av[4 * v + 3] = A.w;
+        }
         dump(c, (kst * KBS) + kb, ra[cur], rb[cur]);
         if constexpr (!EXO) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < KK; ++kk) {
             const float2 u0 = __ffma2_rn(f2(ra[cur][2 * kk], ra[cur][2 * kk + 1]), Wp0, Cp0);
             const float2 u1 = __ffma2_rn(f2(rb[cur][2 * kk], rb[cur][2 * kk + 1]), Wp1, Cp1);
             const float2 ap = make_float2(av[kk], av[kk]);
@@ -461,7 +487,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         } else {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
+          for (int kk = 0; kk < KK; ++kk) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const uint32_t* rr = j ? rb[cur] : ra[cur];
@@ -474,8 +500,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (c + 1 < CHUNKS) {
           if (EXO) {
-            tmem_ld_16x128b_x4(tb + 16u * (c + 1), ra[cur ^ 1]);
-            tmem_ld_16x128b_x4(tb + 16u * (c + 1) + (16u << 16), rb[cur ^ 1]);
+            tmem_ld_chunk(tb + (uint32_t)CW * (c + 1), ra[cur ^ 1]);
+            tmem_ld_chunk(tb + (uint32_t)CW * (c + 1) + (16u << 16), rb[cur ^ 1]);
           }
           tc_wait_ld();
           regs_after_wait(ra[cur ^ 1]);
@@ -502,7 +528,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 2; ++j)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) acc[c][j][kk] = make_float2(0.0f, 0.0f);
+            for (int kk = 0; kk < KK; ++kk) acc[c][j][kk] = make_float2(0.0f, 0.0f);
       }
       using K0 = std::integral_constant<int, 0>;
       using K1 = std::integral_constant<int, 1>;
@@ -523,14 +549,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         // of it) at a time; the row pointer advances by a volatile add so the
         // compiler does not form all the store addresses at once
         const int nr = n0 + q * 32 + l8;
-        const int mr = m0 + h * T::COLS_W + c4;
+        const int mr = m0 + h * COLS_W + c4;
         __nv_bfloat16* p = out + (size_t)mr * (size_t)ldo + nr;
         const long long step = 4 * ldo;
 #pragma unroll
         for (int c = 0; c < CHUNKS; ++c) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int mm = mr + 16 * c + 4 * kk;
+          for (int kk = 0; kk < KK; ++kk) {
+            const int mm = mr + CW * c + 4 * kk;
             if (mm < m) {
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
@@ -554,20 +580,37 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
 }
 
+// Epilogue configuration per tile width: (epilogue warps, chunk columns).
+template <int BM>
+struct Epi;
+template <>
+struct Epi<128> {
+  static constexpr int EW = 8, CW = 32;
+};
+template <>
+struct Epi<192> {
+  static constexpr int EW = 8, CW = 32;
+};
+template <>
+struct Epi<256> {
+  static constexpr int EW = 8, CW = 16;
+};
+
 // Shared-memory opt-in per device and kernel variant, made once under a lock.
 std::mutex g_optin_mu;
 bool g_optin[64][6] = {};
 
 template <int BM, bool DUMP>
 cudaError_t optin_variant(int dev) {
+  constexpr int EW = Epi<BM>::EW, CW = Epi<BM>::CW;
   const int slot = (BM == 128 ? 0 : BM == 192 ? 2 : 4) + (DUMP ? 1 : 0);
   if (g_optin[dev][slot]) return cudaSuccess;
   cudaFuncAttributes fa;
-  cudaError_t e = cudaFuncGetAttributes(&fa, gemm_kernel<BM, DUMP>);
+  cudaError_t e = cudaFuncGetAttributes(&fa, gemm_kernel<BM, EW, CW, DUMP>);
   if (e != cudaSuccess) return e;
   // the register split assumes every thread starts with LAUNCH_REGS registers
-  if (fa.numRegs < LAUNCH_REGS) return cudaErrorInvalidConfiguration;
-  e = cudaFuncSetAttribute(gemm_kernel<BM, DUMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (fa.numRegs < Warps<EW>::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(gemm_kernel<BM, EW, CW, DUMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem_bytes<BM>());
   if (e != cudaSuccess) return e;
   g_optin[dev][slot] = true;
@@ -582,20 +625,23 @@ cudaError_t optin(int dev, bool partials) {
 template <int BM>
 void launch_bm(const GemmMaps& maps, __nv_bfloat16* out, int32_t* partials, int* status, int m, int n, int k,
                long long ldo, cudaStream_t stream, int grid, int n_tiles, int m_tiles, int m_fastest) {
+  constexpr int EW = Epi<BM>::EW, CW = Epi<BM>::CW;
+  constexpr int threads = Warps<EW>::THREADS;
   if (partials)
-    gemm_kernel<BM, true><<<grid, THREADS, smem_bytes<BM>(), stream>>>(
+    gemm_kernel<BM, EW, CW, true><<<grid, threads, smem_bytes<BM>(), stream>>>(
         maps.w, maps.a, maps.ws, maps.as, out, partials, status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
   else
-    gemm_kernel<BM, false><<<grid, THREADS, smem_bytes<BM>(), stream>>>(
+    gemm_kernel<BM, EW, CW, false><<<grid, threads, smem_bytes<BM>(), stream>>>(
         maps.w, maps.a, maps.ws, maps.as, out, nullptr, status, m, n, k, n_tiles, m_tiles, m_fastest, ldo);
 }
 
 // Relative epilogue throughput per element of the tile widths, measured on
 // B200 from whole-kernel times of the three widths on the 2048 x 14336 x
 // 4096, 8192 x 4096 x 14336 and 4095 x 8192 x 8192 projections (they agree
-// within 2%): 192 rows give each thread 96 columns with no register spills;
-// 256 rows need more registers than the epilogue warps hold.
-constexpr double kRate128 = 1.0, kRate192 = 1.10, kRate256 = 0.945;
+// within 2%): 192 rows give each thread 96 columns in three 32-column chunks
+// with no register spills; 256 rows need more registers than the epilogue
+// warps hold.
+constexpr double kRate128 = 1.0, kRate192 = 1.145, kRate256 = 0.945;
 
 }  // namespace gemm
 
