@@ -228,7 +228,10 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
 #pragma unroll
     for (int r = 0; r < MR; ++r) acc[r] = 0.0f;
     for (int b = lane, c = 0; c < (int)L.chunks; b += 32, ++c) {
-      if (!mbar_wait(&bars[c], phase, abort_flag, status, DEV_ERR_TIMEOUT_DECODE)) {
+      // warp-uniform decision: a lane whose wait ran out takes the whole warp
+      // out (the warp synchronises after the row)
+      const bool landed = mbar_wait(&bars[c], phase, abort_flag, status, DEV_ERR_TIMEOUT_DECODE);
+      if (__any_sync(0xFFFFFFFFu, !landed)) {
         aborted = true;
         break;
       }

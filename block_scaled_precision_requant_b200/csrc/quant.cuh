@@ -90,4 +90,81 @@ __device__ __forceinline__ uint2 quant8_quad(const float (&x)[8], float& scale_o
   return make_uint2(pack4_s8(q[0], q[1], q[2], q[3]), pack4_s8(q[4], q[5], q[6], q[7]));
 }
 
+// Four codes in [-127, 127] packed into one word, element 0 in byte 0
+// (two saturating pack conversions; the saturation never binds).
+__device__ __forceinline__ uint32_t pack4_cvt(int q0, int q1, int q2, int q3) {
+  uint32_t hi, d;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(q3), "r"(q2));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(q1), "r"(q0), "r"(hi));
+  return d;
+}
+
+// Largest |x| of 16 BF16 pairs, as float32 (exact).  |x| of a BF16 value is
+// its bit pattern with the sign cleared, and for non-NaN values the order of
+// those patterns as unsigned integers is the order of the magnitudes, so
+// the maximum is taken with packed 16-bit unsigned max operations.
+__device__ __forceinline__ float bf16x32_amax(const uint4 (&v)[4]) {
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    m = __vmaxu2(m, v[i].x & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v[i].y & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v[i].z & 0x7FFF7FFFu);
+    m = __vmaxu2(m, v[i].w & 0x7FFF7FFFu);
+  }
+  const uint32_t hm = (m >> 16) > (m & 0xFFFFu) ? (m >> 16) : (m & 0xFFFFu);
+  return __uint_as_float(hm << 16);
+}
+
+// Code of x for a group with a normal reciprocal (g.rcp != 0): the product
+// by RN(1/scale) rounded half-even, or the rounded IEEE quotient when the
+// product lies within 2^-15 of a half-integer (see the file comment).  The
+// result is in [-127, 127] without a clamp: |y| <= 127 (1 + 2^-23)^2 < 127.5.
+__device__ __forceinline__ int quant_code_rcp(float x, const GroupScale& g) {
+  const float y = __fmul_rn(x, g.rcp);
+  float ry = rintf(y);
+  if (fabsf(__fsub_rn(y, ry)) >= kTieGuard) ry = rintf(__fdiv_rn(x, g.scale));
+  return __float2int_rn(ry);
+}
+
+// One whole 32-group in one thread: 32 BF16 values (four 16-byte loads) ->
+// 32 codes (two 16-byte words) and the group scale.  Same rule as
+// quant_code; all-zero (or underflowing) groups give scale 0 and codes 0.
+__device__ __forceinline__ void quant_group32(const uint4 (&v)[4], uint4& c_lo, uint4& c_hi, float& scale_out) {
+  const GroupScale g = group_scale(bf16x32_amax(v));
+  scale_out = g.scale;
+  uint32_t w[8];
+  if (g.rcp != 0.0f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t p[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int q0 = quant_code_rcp(__uint_as_float(p[2 * j] << 16), g);
+        const int q1 = quant_code_rcp(__uint_as_float(p[2 * j] & 0xFFFF0000u), g);
+        const int q2 = quant_code_rcp(__uint_as_float(p[2 * j + 1] << 16), g);
+        const int q3 = quant_code_rcp(__uint_as_float(p[2 * j + 1] & 0xFFFF0000u), g);
+        w[2 * i + j] = pack4_cvt(q0, q1, q2, q3);
+      }
+    }
+  } else {
+    // scale 0 (all-zero group) or subnormal (every code by exact division)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t p[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        int q[4];
+        const float x[4] = {__uint_as_float(p[2 * j] << 16), __uint_as_float(p[2 * j] & 0xFFFF0000u),
+                            __uint_as_float(p[2 * j + 1] << 16), __uint_as_float(p[2 * j + 1] & 0xFFFF0000u)};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) q[e] = (g.scale == 0.0f) ? 0 : quant_code(x[e], g);
+        w[2 * i + j] = pack4_cvt(q[0], q[1], q[2], q[3]);
+      }
+    }
+  }
+  c_lo = make_uint4(w[0], w[1], w[2], w[3]);
+  c_hi = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
 }  // namespace bsr

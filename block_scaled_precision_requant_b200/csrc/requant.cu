@@ -64,16 +64,22 @@ struct CodeTable {
 __device__ __forceinline__ CodeTable block_codes(float s_e4m3, float scale2, const GroupScale& g) {
   int q[8];
   q[0] = 0;
+  if (g.rcp != 0.0f) {
 #pragma unroll
-  for (int i = 1; i < 8; ++i) {
-    const float v = __fmul_rn(e2m1_mag(i) * s_e4m3, scale2);  // e2m1 * e4m3 is exact
-    q[i] = (g.scale == 0.0f) ? 0 : quant_code(v, g);
+    for (int i = 1; i < 8; ++i)
+      q[i] = quant_code_rcp(__fmul_rn(e2m1_mag(i) * s_e4m3, scale2), g);  // e2m1 * e4m3 is exact
+  } else {
+#pragma unroll
+    for (int i = 1; i < 8; ++i) {
+      const float v = __fmul_rn(e2m1_mag(i) * s_e4m3, scale2);
+      q[i] = (g.scale == 0.0f) ? 0 : quant_code(v, g);
+    }
   }
   CodeTable t;
-  t.pos_lo = pack4_s8(q[0], q[1], q[2], q[3]);
-  t.pos_hi = pack4_s8(q[4], q[5], q[6], q[7]);
-  t.neg_lo = pack4_s8(-q[0], -q[1], -q[2], -q[3]);
-  t.neg_hi = pack4_s8(-q[4], -q[5], -q[6], -q[7]);
+  t.pos_lo = pack4_cvt(q[0], q[1], q[2], q[3]);
+  t.pos_hi = pack4_cvt(q[4], q[5], q[6], q[7]);
+  t.neg_lo = pack4_cvt(-q[0], -q[1], -q[2], -q[3]);
+  t.neg_hi = pack4_cvt(-q[4], -q[5], -q[6], -q[7]);
   return t;
 }
 
@@ -101,7 +107,6 @@ __device__ __forceinline__ uint2 map_word(uint32_t w, const CodeTable& t) {
   return make_uint2((p0 & ~m0) | (n0 & m0), (p1 & ~m1) | (n1 & m1));
 }
 
-constexpr int kUnroll = 4;  // requant_a: tasks per warp and pass, loads first
 
 __global__ void __launch_bounds__(256) requant_w_kernel(const uint4* __restrict__ w_packed,
                                                         const uint16_t* __restrict__ w_e4m3, float scale2,
@@ -131,47 +136,64 @@ __global__ void __launch_bounds__(256) requant_w_kernel(const uint4* __restrict_
 // ---------------------------------------------------------------------------
 // requant_a
 //
-// Four lanes per 32-group (8 BF16 each, one 16-byte load), eight groups per
-// warp taken from eight consecutive rows at the same block b, so the loads
-// are 64-byte row segments, the codes 32-byte segments and the eight scales
-// one 32-byte segment of the block-major scale array.
+// One thread per 32-group: four 16-byte loads (64 contiguous bytes), the
+// amax by packed 16-bit max, the group scale once, 32 codes in two 16-byte
+// stores.  A warp takes 8 consecutive rows x 4 consecutive blocks (lane L:
+// row 8R + L%8, block 4B + L/8), so its loads are eight 256-byte row
+// segments, its codes eight 128-byte segments, and its scales four 32-byte
+// segments of the block-major scale array.  The next task's loads are issued
+// before the current task's arithmetic.
 // ---------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(256) requant_a_kernel(const uint4* __restrict__ a, uint2* __restrict__ a_i8,
+__global__ void __launch_bounds__(256) requant_a_kernel(const uint16_t* __restrict__ a, int8_t* __restrict__ a_i8,
                                                         float* __restrict__ a_scale_t, int m, int k, int ld) {
   const int lane = threadIdx.x & 31;
   const int nb = k >> 5;
-  const long long tasks = (long long)((m + 7) >> 3) * nb;
+  const int nb4 = (nb + 3) >> 2;
+  const long long tasks = (long long)((m + 7) >> 3) * nb4;
   const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  const int sub = lane & 3;
-  // Four tasks per warp and pass, their loads issued before any arithmetic.
-  for (long long t0 = warp0; t0 < tasks; t0 += kUnroll * nwarps) {
-    uint4 v[kUnroll];
-    long long e[kUnroll];
-    int row[kUnroll], blk[kUnroll];
+  auto locate = [&](long long t, int& row, int& blk) {
+    const long long r8 = t / nb4;
+    row = (int)(r8 * 8) + (lane & 7);
+    blk = (int)(t - r8 * nb4) * 4 + (lane >> 3);
+  };
+  auto load = [&](int row, int blk, uint4 (&v)[4]) {
+    if (row < m && blk < nb) {
+      const uint4* src = reinterpret_cast<const uint4*>(a + (size_t)row * k + (size_t)blk * 32);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long long t = t0 + u * nwarps;
-      const int r8 = (int)(t / nb);
-      blk[u] = (int)(t - (long long)r8 * nb);
-      row[u] = r8 * 8 + (lane >> 2);
-      const bool valid = t < tasks && row[u] < m;  // uniform per group of 4 lanes
-      e[u] = valid ? (long long)row[u] * k + (long long)blk[u] * 32 + sub * 8 : -1;
-      v[u] = valid ? __ldg(a + (e[u] >> 3)) : make_uint4(0, 0, 0, 0);
-    }
+      for (int i = 0; i < 4; ++i) v[i] = __ldg(src + i);
+    } else {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (t0 + u * nwarps >= tasks) break;  // uniform per warp
-      float x[8];
-      bf16x8_to_f32(v[u], x);
-      float s;
-      const uint2 c = quant8_quad(x, s);
-      if (e[u] >= 0) {
-        a_i8[e[u] >> 3] = c;
-        if (sub == 0) a_scale_t[(long long)blk[u] * ld + row[u]] = s;
-      }
+      for (int i = 0; i < 4; ++i) v[i] = make_uint4(0, 0, 0, 0);
     }
+  };
+  long long t = warp0;
+  if (t >= tasks) return;
+  int row, blk;
+  locate(t, row, blk);
+  uint4 v[4];
+  load(row, blk, v);
+  for (; t < tasks; t += nwarps) {
+    int nrow = 0, nblk = 0;
+    uint4 nv[4];
+    if (t + nwarps < tasks) {
+      locate(t + nwarps, nrow, nblk);
+      load(nrow, nblk, nv);
+    }
+    uint4 lo, hi;
+    float scale;
+    quant_group32(v, lo, hi, scale);
+    if (row < m && blk < nb) {
+      uint4* dst = reinterpret_cast<uint4*>(a_i8 + (size_t)row * k + (size_t)blk * 32);
+      dst[0] = lo;
+      dst[1] = hi;
+      a_scale_t[(size_t)blk * ld + row] = scale;
+    }
+    row = nrow;
+    blk = nblk;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = nv[i];
   }
 }
 
@@ -198,10 +220,10 @@ cudaError_t launch_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, flo
 
 cudaError_t launch_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, int m, int k, int ld,
                              cudaStream_t stream, int num_sms) {
-  const long long tasks = (long long)((m + 7) / 8) * (k / 32);
+  // warp tasks of 8 rows x 4 blocks, 8 warps per CTA
+  const long long tasks = (long long)((m + 7) / 8) * ((k / 32 + 3) / 4);
   const int grid = grid_for(tasks, 8, num_sms * 8);
-  requant_a_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(a), reinterpret_cast<uint2*>(a_i8),
-                                             a_scale_t, m, k, ld);
+  requant_a_kernel<<<grid, 256, 0, stream>>>(a, a_i8, a_scale_t, m, k, ld);
   return cudaGetLastError();
 }
 

@@ -6,21 +6,24 @@
 //
 //     x = bf16_rne(silu(g) * u),   silu(g) = g / (1 + exp(-g)),
 //
-// every step a float32 operation rounded to nearest (intrinsics, so nothing
-// is contracted into an FMA), and the quantiser is requant_a of x: one F32
-// scale per 32 elements, codes rint(x / scale) clamped to +-127.
+// and the quantiser is requant_a of x (same code as requant_a, so the fused
+// quantiser is bit-identical to the product followed by requant_a).
 //
-// exp is computed by explicit steps (Cody-Waite range reduction with a
-// two-part ln 2 and a degree-6 Taylor polynomial in Horner form), not by the
-// CUDA math library, so that the result is a fixed function of the input:
-//
-//     n = rint(x * log2e)                     (half-even)
-//     r = (x - n * ln2_hi) - n * ln2_lo        (n * ln2_hi exact: ln2_hi has 15 bits)
-//     p = 1 + r(1 + r(1/2 + r(1/6 + r(1/24 + r(1/120 + r/720)))))
-//     exp(x) = (p * 2^h1) * 2^h2,  h1 = floor(n/2), h2 = n - h1
-//
-// with x > 88 -> +inf and x < -88 -> +0.  Over [-88, 88] it is within 3 ulp
-// of exp.
+// The kernel evaluates silu(g) without overflow for either sign of g, with
+// t = exp(-|g|) in (0, 1]:
+//     silu(g) = g / (1 + t)        for g >= 0,
+//     silu(g) = (g * t) / (1 + t)  for g < 0,
+// and exp by Cody-Waite range reduction with a two-part ln 2 followed by the
+// hardware base-2 exponential of the reduced argument:
+//     n = rint(x * log2e),  r = (x - n * ln2_hi) - n * ln2_lo,  |r| <= ln2/2
+//     exp(x) = 2^(r * log2e) * 2^n           (x = -|g| <= 0)
+// The reduced argument keeps the hardware's relative error (about 2^-22) for
+// every |g|; with the approximate quotient (2 ulp) and three roundings the
+// float32 product is within 2^-20 of the exact silu(g) * u, so its BF16
+// rounding equals the exact product's except within 2^-20 of a rounding
+// boundary.  For g < -104 the kernel takes t = 0 (e^-104 is below float32's
+// range), so its product is a signed zero; the exact product rounds to zero
+// in BF16 there unless |u| > 650.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -32,39 +35,36 @@ namespace bsr {
 namespace {
 
 constexpr uint32_t kLog2e = 0x3FB8AA3Bu;  // 1.442695f
-constexpr uint32_t kLn2Hi = 0x3F317200u;  // 0.693145751953125f
+constexpr uint32_t kLn2Hi = 0x3F317200u;  // 0.693145751953125f (15 significant bits: n * ln2_hi is exact)
 constexpr uint32_t kLn2Lo = 0x35BFBE8Eu;  // ln 2 - kLn2Hi
-// 1/i! for i = 0..6
-constexpr uint32_t kC0 = 0x3F800000u, kC1 = 0x3F800000u, kC2 = 0x3F000000u, kC3 = 0x3E2AAAABu,
-                   kC4 = 0x3D2AAAABu, kC5 = 0x3C088889u, kC6 = 0x3AB60B61u;
 
-__device__ __forceinline__ float pow2i(int h) {  // 2^h, h in [-126, 127]
-  return __uint_as_float((uint32_t)(h + 127) << 23);
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
-__device__ __forceinline__ float exp_steps(float x) {
-  if (x != x) return x;
-  if (x > 88.0f) return __uint_as_float(0x7F800000u);
-  if (x < -88.0f) return 0.0f;
+// exp(x) for -104 <= x <= 0 (below -126 ln 2 the two-step scaling by
+// 2^h1 * 2^h2 reaches the subnormal range)
+__device__ __forceinline__ float exp_nonpos(float x) {
   const float n = rintf(__fmul_rn(x, __uint_as_float(kLog2e)));
-  const float r = __fsub_rn(__fsub_rn(x, __fmul_rn(n, __uint_as_float(kLn2Hi))), __fmul_rn(n, __uint_as_float(kLn2Lo)));
-  float p = __uint_as_float(kC6);
-  p = __fadd_rn(__fmul_rn(p, r), __uint_as_float(kC5));
-  p = __fadd_rn(__fmul_rn(p, r), __uint_as_float(kC4));
-  p = __fadd_rn(__fmul_rn(p, r), __uint_as_float(kC3));
-  p = __fadd_rn(__fmul_rn(p, r), __uint_as_float(kC2));
-  p = __fadd_rn(__fmul_rn(p, r), __uint_as_float(kC1));
-  p = __fadd_rn(__fmul_rn(p, r), __uint_as_float(kC0));
-  const int ni = (int)n;
-  const int h1 = ni >> 1;  // floor(n / 2)
-  const int h2 = ni - h1;
-  return __fmul_rn(__fmul_rn(p, pow2i(h1)), pow2i(h2));
+  float r = __fmaf_rn(-n, __uint_as_float(kLn2Hi), x);
+  r = __fmaf_rn(-n, __uint_as_float(kLn2Lo), r);
+  const float p = ex2_approx(__fmul_rn(r, __uint_as_float(kLog2e)));
+  const int ni = (int)n;                      // in [-150, 0]
+  const int h1 = ni >= -126 ? ni : -126;      // 2^h1 normal
+  const int h2 = ni - h1;                     // in [-25, 0]
+  const float s1 = __uint_as_float((uint32_t)(h1 + 127) << 23);
+  const float s2 = __uint_as_float((uint32_t)(h2 + 127) << 23);
+  return __fmul_rn(__fmul_rn(p, s1), s2);
 }
 
-// bf16(silu(g) * u) as its float32 value (exact) and its bit pattern
+// bf16(silu(g) * u) as its float32 value (exact)
 __device__ __forceinline__ float silu_mul_value(float g, float u) {
-  const float e = exp_steps(-g);
-  const float s = __fdiv_rn(g, __fadd_rn(1.0f, e));
+  const float ag = fabsf(g);
+  const float t = ag <= 104.0f ? exp_nonpos(-ag) : 0.0f;
+  const float num = g >= 0.0f ? g : __fmul_rn(g, t);
+  const float s = __fdividef(num, __fadd_rn(1.0f, t));
   return __bfloat162float(__float2bfloat16_rn(__fmul_rn(s, u)));
 }
 
@@ -93,36 +93,46 @@ __global__ void __launch_bounds__(256) silu_mul_kernel(const uint4* __restrict__
 }
 
 // requant_a of bf16(silu(g) * u) without writing the product: the task
-// layout of requant_a (four lanes per 32-group, eight rows per warp at one
-// block, block-major scales), with the product formed after the loads.
-__global__ void __launch_bounds__(256) requant_silu_a_kernel(const uint4* __restrict__ g, const uint4* __restrict__ u,
-                                                             uint2* __restrict__ a_i8, float* __restrict__ a_scale_t,
+// layout of requant_a (one thread per 32-group, a warp on 8 rows x 4
+// blocks, block-major scales), the 32 products formed after the loads and
+// quantised by the same code as requant_a.
+__global__ void __launch_bounds__(256) requant_silu_a_kernel(const uint16_t* __restrict__ g,
+                                                             const uint16_t* __restrict__ u,
+                                                             int8_t* __restrict__ a_i8, float* __restrict__ a_scale_t,
                                                              int m, int k, int ld) {
   const int lane = threadIdx.x & 31;
   const int nb = k >> 5;
-  const long long tasks = (long long)((m + 7) >> 3) * nb;
-  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nb4 = (nb + 3) >> 2;
+  const long long tasks = (long long)((m + 7) >> 3) * nb4;
   const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
-  const int sub = lane & 3;
-  for (long long t = warp0; t < tasks; t += nwarps) {
-    const int r8 = (int)(t / nb);
-    const int b = (int)(t - (long long)r8 * nb);
-    const int row = r8 * 8 + (lane >> 2);
-    const bool valid = row < m;  // uniform per group of 4 lanes
-    const long long e = (long long)(valid ? row : 0) * k + (long long)b * 32 + sub * 8;
-    uint4 gv = make_uint4(0, 0, 0, 0), uv = make_uint4(0, 0, 0, 0);
-    if (valid) {
-      gv = __ldg(g + (e >> 3));
-      uv = __ldg(u + (e >> 3));
+  for (long long t = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < tasks; t += nwarps) {
+    const long long r8 = t / nb4;
+    const int row = (int)(r8 * 8) + (lane & 7);
+    const int blk = (int)(t - r8 * nb4) * 4 + (lane >> 3);
+    if (row >= m || blk >= nb) continue;  // no warp-wide operation below
+    const size_t off = (size_t)row * k + (size_t)blk * 32;
+    const uint4* gs = reinterpret_cast<const uint4*>(g + off);
+    const uint4* us = reinterpret_cast<const uint4*>(u + off);
+    uint4 gv[4], uv[4], v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      gv[i] = __ldg(gs + i);
+      uv[i] = __ldg(us + i);
     }
-    float x[8];
-    silu_mul8(gv, uv, x);
-    float s;
-    const uint2 c = quant8_quad(x, s);
-    if (valid) {
-      a_i8[e >> 3] = c;
-      if (sub == 0) a_scale_t[(long long)b * ld + row] = s;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float x[8];
+      silu_mul8(gv[i], uv[i], x);
+      v[i] = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                        pack_bf16x2(x[6], x[7]));
     }
+    uint4 lo, hi;
+    float scale;
+    quant_group32(v, lo, hi, scale);
+    uint4* dst = reinterpret_cast<uint4*>(a_i8 + off);
+    dst[0] = lo;
+    dst[1] = hi;
+    a_scale_t[(size_t)blk * ld + row] = scale;
   }
 }
 
@@ -146,11 +156,9 @@ cudaError_t launch_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* x, i
 
 cudaError_t launch_requant_silu_a(const uint16_t* g, const uint16_t* u, int8_t* a_i8, float* a_scale_t, int m, int k,
                                   int ld, cudaStream_t stream, int num_sms) {
-  const long long tasks = (long long)((m + 7) / 8) * (k / 32);
+  const long long tasks = (long long)((m + 7) / 8) * ((k / 32 + 3) / 4);
   const int grid = grid_for(tasks, 8, num_sms * 8);
-  requant_silu_a_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(g),
-                                                  reinterpret_cast<const uint4*>(u), reinterpret_cast<uint2*>(a_i8),
-                                                  a_scale_t, m, k, ld);
+  requant_silu_a_kernel<<<grid, 256, 0, stream>>>(g, u, a_i8, a_scale_t, m, k, ld);
   return cudaGetLastError();
 }
 

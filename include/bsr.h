@@ -316,10 +316,13 @@ bsr_status bsr_w4a4_proj(const uint16_t* a, const uint8_t* w_packed, const uint8
  * SiLU.mul quantiser for the down projection (w8a8_decode/parts.rs names it,
  * `W8a8Kernels::quant_silu`; the pages give no arithmetic).  Reading taken:
  *   x = bf16_rne(silu(g) * u),  silu(g) = g / (1 + exp(-g)),
- * each step a float32 operation rounded to nearest, exp by fixed steps
- * (Cody-Waite reduction, degree-6 Taylor polynomial; within 3 ulp of exp on
- * [-88, 88], +inf above 88, +0 below -88).  Inputs gate, up: [M, K] BF16,
- * finite.  Requirements and errors as bsr_requant_a.
+ * the exact product rounded once to BF16.  The kernels evaluate it in
+ * float32 (exp of -|g| by range reduction and the hardware base-2
+ * exponential, an approximate quotient) within 2^-20 relative of the exact
+ * product, so x equals the exact rounding except within 2^-20 of a BF16
+ * rounding boundary (one BF16 step there); for g < -104 x is a signed zero.
+ * Inputs gate, up: [M, K] BF16, finite.  Requirements and errors as
+ * bsr_requant_a.
  */
 
 /* x [M, K] BF16 out: the product itself (the unfused activation). */
