@@ -64,6 +64,9 @@ def parse_args(argv=None):
     p.add_argument("--no-extra", action="store_true", help="skip the secondary prefill measurements")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline (profiling runs)")
+    p.add_argument("--only", default=None,
+                   choices=["decode", "proj", "gemm", "requant_a", "requant_w", "requant_silu_a"],
+                   help="time one operation of the path alone on the workload (for profiling) and print its line")
     return p.parse_args(argv)
 
 
@@ -1184,10 +1187,53 @@ def gpu_main(args):
     return 0
 
 
+def only_main(args):
+    """One operation of the path alone on the workload, K timed launches
+    after W warm-up launches (L2 flushed before each): a short, predictable
+    launch sequence for profilers.  Prints its time and throughput."""
+    import torch
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    g = Gpu(args.workload, dev)
+    bsr = g.bsr
+    m, n, k = g.wl.shape
+    op = args.only
+    if op == "decode":
+        fn = lambda: bsr.decode(g.a, g.w_i8, g.w_s, g.out)  # noqa: E731
+        units, unit = decode_bytes(m, n, k) / 1e9, "GB/s"
+    elif op == "proj":
+        fn, units, unit = g.step, prefill_ops(m, n, k) / 1e12, "TOPS"
+    elif op == "gemm":
+        fn = lambda: bsr.gemm(g.a_i8, g.a_st, g.w_i8, g.w_s, g.out)  # noqa: E731
+        units, unit = prefill_ops(m, n, k) / 1e12, "TOPS"
+    elif op == "requant_a":
+        fn = lambda: bsr.requant_a(g.a, g.a_i8, g.a_st)  # noqa: E731
+        units, unit = m * k * 3.125 / 1e9, "GB/s"
+    elif op == "requant_w":
+        fn = lambda: bsr.requant_w(g.wp, g.we, float(g.host["scale2"]), g.w_i8, g.w_s)  # noqa: E731
+        units, unit = n * k * 1.6875 / 1e9, "GB/s"
+    else:
+        from block_scaled_precision_requant_b200 import synth
+
+        gb, ub, _ = synth.make_gate_up(m, k, g.wl.seed)
+        gate = torch.from_numpy(gb.view(np.int16)).view(torch.bfloat16).to(dev)
+        up = torch.from_numpy(ub.view(np.int16)).view(torch.bfloat16).to(dev)
+        fn = lambda: bsr.requant_silu_a(gate, up, g.a_i8, g.a_st)  # noqa: E731
+        units, unit = m * k * 5.125 / 1e9, "GB/s"
+    ms = mean_ms(g.timed(fn, args.steps, args.warmup))
+    g.check_status()
+    print(json.dumps({"only": op, "workload": g.wl.name, "ms": ms, "value": units / (ms / 1e3), "unit": unit,
+                      "steps": args.steps, "warmup": args.warmup}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return reference_main(args)
+    if args.only:
+        return only_main(args)
     return gpu_main(args)
 
 
