@@ -65,7 +65,7 @@ def parse_args(argv=None):
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the oracle baseline sample")
     p.add_argument("--no-cpu", action="store_true", help="skip the oracle baseline (profiling runs)")
     p.add_argument("--only", default=None,
-                   choices=["decode", "proj", "gemm", "requant_a", "requant_w", "requant_silu_a"],
+                   choices=["decode", "proj", "gemm", "requant_a", "requant_w", "requant_silu_a", "w4a16", "w4a4_decode"],
                    help="time one operation of the path alone on the workload (for profiling) and print its line")
     return p.parse_args(argv)
 
@@ -792,7 +792,8 @@ def w4a4_gemm_extra(device, steps, warmup, peaks):
             "gemm_tops": ops / t_gemm / 1e9, "ms_gemm": t_gemm,
             "fp4_peak": fp4_peak, "gemm_frac_of_fp4_peak": ops / t_gemm / 1e9 / fp4_peak,
             "peak_source": f"measured bf16 burst x {FP4_PER_BF16:g} (nominal dense FP4/bf16 ratio)",
-            "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
+            "static_weight": True,
+           "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
 
 
 def stacked_decode_extra(device, steps, peaks, cpu=True):
@@ -878,12 +879,12 @@ def w4a16_extra(g, steps, peaks, cpu=True):
     s2 = float(g.host["scale2"])
     out = torch.empty((m, n), dtype=torch.bfloat16, device=g.dev)
     for i in range(3):
-        bsr.w4a16_decode(g.a, *ws[i % copies], s2, out)
+        bsr.w4a16_decode(g.a, *ws[i % copies], s2, out, static_weight=True)
     torch.cuda.synchronize()
     gr = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gr):
         for i in range(steps):
-            bsr.w4a16_decode(g.a, *ws[i % copies], s2, out)
+            bsr.w4a16_decode(g.a, *ws[i % copies], s2, out, static_weight=True)
     gr.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -896,6 +897,7 @@ def w4a16_extra(g, steps, peaks, cpu=True):
     g.check_status()
     res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
            "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "static_weight": True,
            "note": "reads the NVFP4 weight as stored; not bit-compatible with the int8 path"}
     if cpu:
         import oracle
@@ -938,12 +940,12 @@ def w4a4_extra(device, wl, host, steps, peaks, cpu=True):
     s2 = float(host["scale2"])
     out = torch.empty((m, n), dtype=torch.bfloat16, device=device)
     for i in range(3):
-        bsr.w4a4_decode(a, *ws[i % copies], s2, out)
+        bsr.w4a4_decode(a, *ws[i % copies], s2, out, static_weight=True)
     torch.cuda.synchronize()
     gr = torch.cuda.CUDAGraph()
     with torch.cuda.graph(gr):
         for i in range(steps):
-            bsr.w4a4_decode(a, *ws[i % copies], s2, out)
+            bsr.w4a4_decode(a, *ws[i % copies], s2, out, static_weight=True)
     gr.replay()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -957,6 +959,7 @@ def w4a4_extra(device, wl, host, steps, peaks, cpu=True):
         raise RuntimeError(f"device status word {bsr.device_status()}")
     res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
            "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+           "static_weight": True,
            "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
     if cpu:
         import oracle
@@ -1213,6 +1216,11 @@ def only_main(args):
     elif op == "requant_w":
         fn = lambda: bsr.requant_w(g.wp, g.we, float(g.host["scale2"]), g.w_i8, g.w_s)  # noqa: E731
         units, unit = n * k * 1.6875 / 1e9, "GB/s"
+    elif op in ("w4a16", "w4a4_decode"):
+        call = bsr.w4a16_decode if op == "w4a16" else bsr.w4a4_decode
+        s2 = float(g.host["scale2"])
+        fn = lambda: call(g.a, g.wp, g.we, s2, g.out)  # noqa: E731
+        units, unit = (n * k // 2 + n * k // 16 + 2 * m * k + 2 * m * n) / 1e9, "GB/s"
     else:
         from block_scaled_precision_requant_b200 import synth
 

@@ -104,8 +104,10 @@ SIGNATURES = [
     ("bsr_decode_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_proj_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_w4a16_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
+    ("bsr_w4a16_decode_ex", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_nvfp4_quant_rows", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     ("bsr_w4a4_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
+    ("bsr_w4a4_decode_ex", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_nvfp4_sf_blocked_bytes", ctypes.c_size_t, [_I64, _I64]),
     ("bsr_nvfp4_sf_blocked", ctypes.c_int, [_P, _P, _I64, _I64, _P]),
     ("bsr_w4a4_gemm", ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P, _P]),
@@ -513,15 +515,14 @@ def proj_stacked(a, segments, out=None, scratch=None, stream=None):
     return out
 
 
-def w4a16_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
-    """NVFP4 W4A16 decode GEMV on the stored weight -> out [M, N] bfloat16."""
+def _nvfp4_gemv(entry, a, w_packed, w_e4m3, scale2, out, stream, static_weight):
     torch = _torch()
     m, k = a.shape
     n = w_packed.shape[0]
     if out is None:
         out = _empty((m, n), torch.bfloat16, a)
     _check(
-        lib().bsr_w4a16_decode(
+        entry(
             _dev(a, torch.bfloat16, (m, k), "a"),
             _dev(w_packed, torch.uint8, (n, k // 2), "w_packed"),
             _dev(w_e4m3, torch.uint8, (n, k // 16), "w_e4m3"),
@@ -530,10 +531,17 @@ def w4a16_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
             m,
             n,
             k,
+            DECODE_STATIC_WEIGHT if static_weight else 0,
             _stream_ptr(stream),
         )
     )
     return out
+
+
+def w4a16_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None, static_weight=False):
+    """NVFP4 W4A16 decode GEMV on the stored weight -> out [M, N] bfloat16.
+    ``static_weight=True`` as in :func:`decode`."""
+    return _nvfp4_gemv(lib().bsr_w4a16_decode_ex, a, w_packed, w_e4m3, scale2, out, stream, static_weight)
 
 
 def quant_nvfp4_rows(a, out=None, stream=None):
@@ -559,28 +567,11 @@ def quant_nvfp4_rows(a, out=None, stream=None):
     return packed, e4, s2
 
 
-def w4a4_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None):
+def w4a4_decode(a, w_packed, w_e4m3, scale2: float, out=None, stream=None, static_weight=False):
     """NVFP4 W4A4 decode GEMV (activation rows quantised to NVFP4 inside the
-    kernel) -> out [M, N] bfloat16."""
-    torch = _torch()
-    m, k = a.shape
-    n = w_packed.shape[0]
-    if out is None:
-        out = _empty((m, n), torch.bfloat16, a)
-    _check(
-        lib().bsr_w4a4_decode(
-            _dev(a, torch.bfloat16, (m, k), "a"),
-            _dev(w_packed, torch.uint8, (n, k // 2), "w_packed"),
-            _dev(w_e4m3, torch.uint8, (n, k // 16), "w_e4m3"),
-            ctypes.c_float(float(scale2)),
-            _dev(out, torch.bfloat16, (m, n), "out"),
-            m,
-            n,
-            k,
-            _stream_ptr(stream),
-        )
-    )
-    return out
+    kernel) -> out [M, N] bfloat16.  ``static_weight=True`` as in
+    :func:`decode`."""
+    return _nvfp4_gemv(lib().bsr_w4a4_decode_ex, a, w_packed, w_e4m3, scale2, out, stream, static_weight)
 
 
 def sf_blocked_bytes(rows: int, k: int) -> int:

@@ -18,9 +18,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbsr.so")
-SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "w4a16.cu",
+SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "nvfp4_gemv.cu",
            "w4a4.cu", "w4a4_gemm.cu"]
-HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh", "w4a4_desc.cuh"]
+HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh", "w4a4_desc.cuh", "fp_cvt.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -36,6 +36,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct DevInfo {
   int num_sms = 0;
   size_t smem_optin = 0;
+  size_t smem_per_sm = 0;
   int cc_major = 0;
   int* status = nullptr;  // device address of g_dev_status
 };
@@ -51,9 +52,10 @@ bsr_status device_info(DevInfo& out) {
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DevInfo& d = g_dev[dev];
   if (d.num_sms == 0) {
-    int sms = 0, smem = 0, major = 0;
+    int sms = 0, smem = 0, smem_sm = 0, major = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess ||
         (e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
       return fail(BSR_ENODEV, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
     void* st = nullptr;
@@ -61,6 +63,7 @@ bsr_status device_info(DevInfo& out) {
       return fail(BSR_ENODEV, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     d.num_sms = sms;
     d.smem_optin = (size_t)smem;
+    d.smem_per_sm = (size_t)smem_sm;
     d.cc_major = major;
     d.status = static_cast<int*>(st);
   }
@@ -570,21 +573,29 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
   return ok();
 }
 
-bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
-                            uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream) {
+bsr_status bsr_w4a16_decode_ex(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                               uint16_t* out, int64_t m, int64_t n, int64_t k, unsigned flags, void* stream) {
   bsr_status st = check_dims(m, n, k, true, true);
   if (st != BSR_OK) return st;
+  if (flags & ~BSR_DECODE_STATIC_WEIGHT) return fail(BSR_EINVAL, "unknown flags 0x%x", flags);
   if (m == 0 || n == 0) return ok();
   if (!a || !w_packed || !w_e4m3 || !out) return fail(BSR_EINVAL, "null pointer");
   if (!aligned16(a) || !aligned16(w_packed) || !aligned16(w_e4m3) || (reinterpret_cast<uintptr_t>(out) & 1u))
     return fail(BSR_EALIGN, "a, w_packed, w_e4m3 must be 16-byte aligned, out 2-byte aligned");
   DevInfo d;
   if ((st = device_info(d)) != BSR_OK) return st;
-  if ((size_t)k * 2 > d.smem_optin)
-    return fail(BSR_ESHAPE, "K=%lld too large for one BF16 activation row in shared memory", (long long)k);
-  return cuda_status(bsr::launch_w4a16_decode(a, w_packed, w_e4m3, scale2, out, (int)m, (int)n, (int)k, d.smem_optin,
-                                              as_stream(stream), d.num_sms),
+  bsr::GemvPlan p;
+  if (!bsr::nvfp4_gemv_plan((int)m, (int)n, (int)k, false, d.smem_optin, d.smem_per_sm, d.num_sms, p))
+    return fail(BSR_ESHAPE, "K=%lld, M=%lld outside the NVFP4 GEMV (K <= 65536 with one activation row and one weight stage in shared memory)",
+                (long long)k, (long long)m);
+  return cuda_status(bsr::launch_nvfp4_gemv(p, false, a, w_packed, w_e4m3, scale2, out, (int)m, (int)n, (int)k,
+                                            (flags & BSR_DECODE_STATIC_WEIGHT) ? 1 : 0, d.status, as_stream(stream)),
                      "w4a16 decode launch");
+}
+
+bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                            uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream) {
+  return bsr_w4a16_decode_ex(a, w_packed, w_e4m3, scale2, out, m, n, k, 0u, stream);
 }
 
 }  // extern "C"

@@ -62,10 +62,23 @@ cudaError_t launch_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* x, i
 cudaError_t launch_requant_silu_a(const uint16_t* g, const uint16_t* u, int8_t* a_i8, float* a_scale_t, int m, int k,
                                   int ld, cudaStream_t stream, int num_sms);
 
-// NVFP4 W4A16 decode GEMV: out [M, N] = A [M, K] . dequant(W)^T, F32 sums.
-cudaError_t launch_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
-                                uint16_t* out, int m, int n, int k, size_t smem_limit, cudaStream_t stream,
-                                int num_sms);
+// NVFP4 decode GEMVs on the weight as stored (W4A16: BF16 activations; W4A4:
+// activation rows quantised to NVFP4 inside the kernel).  The plan fixes the
+// launch: MR activation rows per CTA (gy = ceil(M / MR) CTA rows),
+// rows_per_cta weight rows per CTA (gx CTAs) in stages of RS rows, `warps`
+// warps taking alternate stages through `slots` slots each (bulk copies when
+// K % 256 == 0).  False if K > 65536, if even one slot per warp does not fit
+// in smem_limit, or if M needs more than 65535 CTA rows.
+struct GemvPlan {
+  int mr, rs, warps, slots, rows_per_cta, gx, gy;
+  size_t smem;
+  bool bulk;
+};
+bool nvfp4_gemv_plan(int m, int n, int k, bool a4, size_t smem_limit, size_t smem_per_sm, int num_sms,
+                     GemvPlan& p);
+cudaError_t launch_nvfp4_gemv(const GemvPlan& p, bool a4, const uint16_t* a, const uint8_t* w_packed,
+                              const uint8_t* w_e4m3, float scale2, uint16_t* out, int m, int n, int k,
+                              int static_weight, int* status, cudaStream_t stream);
 
 // Test entry: one CTA waits on an mbarrier nothing arrives on, through the
 // bounded wait of the pipelined kernels, for at most limit_ns.

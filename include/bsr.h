@@ -222,13 +222,26 @@ bsr_status bsr_proj_stacked(const uint16_t* a, const int8_t* const* w_i8, const 
  *   w_e4m3    [N, K/16] uint8, E4M3 scale of each 16-element block
  *   scale2    per-tensor F32 scale (host value)
  *   out       [M, N]    BF16: sum_k a * (e2m1 * e4m3) * scale2, float32 sums
- * (per 16-block, then times the E4M3 scale, scale2 once at the end).  Not
- * bit-compatible with bsr_proj (that path requantises to int8).  K > 0,
- * K % 32 == 0, 2K bytes within the device's shared memory per CTA; pointers
- * 16-byte aligned (out 2-byte).  Any M; built for M <= 16.
+ * (per 16-block p = the 16 products summed in element order, then
+ * acc = fma(p, e4m3, acc), scale2 once at the end; the blocks of a row are
+ * summed in an order that depends on K only, so an output's bits depend
+ * only on K and its own row and column).  Elements more than 2^32 below the
+ * largest magnitude of their 16-block are rounded to the half-precision
+ * subnormal grid (2^-24 relative to a block scaled into [2^15, 2^16)).  Not
+ * bit-compatible with bsr_proj (that path requantises to int8).
+ * 0 < K <= 65536, K % 32 == 0; pointers 16-byte aligned (out 2-byte); any M
+ * up to 4 * 65535 (built for M <= 16).  Weight rows stream through shared
+ * memory by bulk copies when K % 256 == 0, else are read from global memory.
  */
 bsr_status bsr_w4a16_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
                             uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
+
+/* bsr_w4a16_decode with flags (0 or BSR_DECODE_STATIC_WEIGHT: no kernel that
+ * writes w_packed or w_e4m3 is in flight or queued ahead on the stream; the
+ * kernel then issues its weight copies before waiting for the previous
+ * kernel on the stream).  Same results and errors. */
+bsr_status bsr_w4a16_decode_ex(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                               uint16_t* out, int64_t m, int64_t n, int64_t k, unsigned flags, void* stream);
 
 /*
  * NVFP4 W4A4 (w4a4_proj/fixed.rs, `nvfp4_proj_mx`: a per-row NVFP4 quantiser
@@ -252,15 +265,19 @@ bsr_status bsr_nvfp4_quant_rows(const uint16_t* a, uint8_t* a_packed, uint8_t* a
                                 int64_t k, void* stream);
 
 /* The W4A4 decode GEMV, the quantiser fused in (each CTA quantises its rows
- * of A into shared memory): a [M, K] BF16, w_packed [N, K/2], w_e4m3
- * [N, K/16], scale2 the weight's F32 scale (host value), out [M, N] BF16.
- * The products of a 16-block are exact, the sum over blocks is float32:
- * results agree with the exact product within the BF16 tolerance, and a
- * row's bits do not depend on M or on the other rows.  Any M (built for
- * M <= 16); the quantised rows of up to 16 rows, K * 0.5625 + 4 bytes
- * each, must fit in the device's shared memory per CTA (BSR_ESHAPE). */
+ * of A): a [M, K] BF16, w_packed [N, K/2], w_e4m3 [N, K/16], scale2 the
+ * weight's F32 scale (host value), out [M, N] BF16.  The products of a
+ * 16-block are exact, the sum over blocks is float32 in an order that
+ * depends on K only: results agree with the exact product within the BF16
+ * tolerance, and an output's bits depend only on K and its own row and
+ * column (not on M, N or the other rows).  0 < K <= 65536, K % 16 == 0; any
+ * M up to 4 * 65535 (built for M <= 16). */
 bsr_status bsr_w4a4_decode(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
                            uint16_t* out, int64_t m, int64_t n, int64_t k, void* stream);
+
+/* bsr_w4a4_decode with flags (as bsr_w4a16_decode_ex). */
+bsr_status bsr_w4a4_decode_ex(const uint16_t* a, const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2,
+                              uint16_t* out, int64_t m, int64_t n, int64_t k, unsigned flags, void* stream);
 
 /*
  * W4A4 on the tensor cores (block-scaled FP4 MMA, kind::mxf4nvf4): the same

@@ -112,6 +112,16 @@ def test_decode_ex_rejects_unknown_flags(L):
     assert "flags" in bsr.last_error()
 
 
+def test_nvfp4_gemv_ex_argument_errors(L):
+    f = ctypes.c_float(1.0)
+    for entry in (L.bsr_w4a16_decode_ex, L.bsr_w4a4_decode_ex):
+        assert entry(_fake(256), _fake(256), _fake(256), f, _fake(256), 1, 8, 64, 2, None) == 1
+        assert "flags" in bsr.last_error()
+        assert entry(None, None, None, f, None, 0, 8, 64, 1, None) == 0
+    assert L.bsr_w4a16_decode_ex(_fake(256), _fake(256), _fake(256), f, _fake(256), 1, 8, 48, 0, None) == 3
+    assert L.bsr_w4a16_decode_ex(_fake(264), _fake(256), _fake(256), f, _fake(256), 1, 8, 64, 1, None) == 2
+
+
 def test_stacked_argument_errors(L):
     arr = (ctypes.c_void_p * 1)(_fake(256).value)
     n1 = (ctypes.c_int64 * 1)(8)

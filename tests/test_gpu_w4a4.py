@@ -127,3 +127,24 @@ def test_scale_relayout_to_blocked(rows, k):
     torch.cuda.synchronize()
     assert got.numel() == bsr.sf_blocked_bytes(rows, k)
     assert np.array_equal(got.cpu().numpy(), _blocked_reference(e4, rows, k))
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 300, 8192), (3, 130, 8192), (1, 260, 14336), (2, 100, 20480),
+                                   (1, 36, 53248), (6, 300, 4096), (1, 14336, 4096)])
+def test_w4a4_lane_layouts(m, n, k):
+    # one case per (activation rows per CTA, blocks per lane, warps) variant,
+    # the K = 53248 one with a single-stage ring, the last with ring refills
+    got, w, a_bits = _run(m, n, k, seed=150 + m)
+    ref = oracle.w4a4_proj(a_bits, w["w_packed"], w["w_e4m3"], w["scale2"], k)
+    assert_close_bf16(got, ref, f"w4a4 m={m} n={n} k={k}")
+    assert bsr.device_status() == 0
+
+
+def test_w4a4_bits_independent_of_n_and_static_flag():
+    m, n, k = 3, 600, 4096
+    got, w, a_bits = _run(m, n, k, seed=160)
+    a, wp, we, s2 = up_bf16(a_bits), up_u8(w["w_packed"]), up_u8(w["w_e4m3"]), float(w["scale2"])
+    assert np.array_equal(bf16_bits(bsr.w4a4_decode(a, wp, we, s2, static_weight=True)), got)
+    part = bf16_bits(bsr.w4a4_decode(a, wp[100:357], we[100:357], s2))  # other N, other CTA ranges
+    assert np.array_equal(part, got[:, 100:357])
+    assert bsr.device_status() == 0
