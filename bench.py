@@ -264,7 +264,8 @@ def roofline(bound, achieved, peak, unit, traffic):
 # and the C-ABI layer that picks its launch parameters, these are the sources
 # its DRAM traffic depends on
 KERNEL_UNITS = {"decode_kernel": "decode.cu", "gemm_kernel": "gemm_tc.cu", "requant_a_kernel": "requant.cu",
-                "requant_w_kernel": "requant.cu", "requant_silu_a_kernel": "silu.cu"}
+                "requant_w_kernel": "requant.cu", "requant_silu_a_kernel": "silu.cu",
+                "nvfp4_gemv_kernel": ("nvfp4_gemv.cu", "w4a4.cu")}
 LAUNCH_LAYER = "api.cu"
 
 
@@ -277,7 +278,8 @@ def kernel_sources(kernel: str):
     its translation unit, the launch layer, and every csrc header they
     include, transitively."""
     csrc = _csrc_dir()
-    todo = [KERNEL_UNITS[kernel], LAUNCH_LAYER]
+    unit = KERNEL_UNITS[kernel]
+    todo = [*(unit if isinstance(unit, tuple) else (unit,)), LAUNCH_LAYER]
     seen = set()
     while todo:
         name = todo.pop()
@@ -897,7 +899,7 @@ def w4a16_extra(g, steps, peaks, cpu=True):
     g.check_status()
     res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
            "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-           "static_weight": True,
+           "traffic": stored_traffic("nvfp4_gemv_kernel", "decode_w4a16"), "static_weight": True,
            "note": "reads the NVFP4 weight as stored; not bit-compatible with the int8 path"}
     if cpu:
         import oracle
@@ -959,7 +961,7 @@ def w4a4_extra(device, wl, host, steps, peaks, cpu=True):
         raise RuntimeError(f"device status word {bsr.device_status()}")
     res = {"ms": ms, "gbs": nbytes / (ms / 1e3) / 1e9, "bytes_per_step": nbytes,
            "frac_of_hbm": nbytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
-           "static_weight": True,
+           "traffic": stored_traffic("nvfp4_gemv_kernel", "decode_w4a4"), "static_weight": True,
            "note": "NVFP4 activations and weight; not bit-compatible with the int8 path"}
     if cpu:
         import oracle

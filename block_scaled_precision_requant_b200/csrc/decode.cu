@@ -10,10 +10,10 @@
 //
 // Memory: one warp per weight row.  Lane 0 of each warp streams its row
 // (and, when the row pitch allows, the row's scales) into the warp's own
-// shared-memory slot as 1 KB bulk copies, each completing on its own
-// mbarrier, all issued at kernel start: the whole weight is in flight at
-// once without holding registers, and a warp consumes its first chunks while
-// the rest still stream.  Meanwhile the CTA requantises the activation rows
+// shared-memory slot as bulk copies of up to 16 KB, all issued at kernel
+// start: the whole weight is in flight at once without holding registers.
+// The slot is read in 1 KB chunks, one 32-block per lane, each chunk with
+// its own mbarrier.  Meanwhile the CTA requantises the activation rows
 // into shared memory (same rule and code as requant_a, so the codes match it
 // bit for bit).  Launched with programmatic dependent launch: activations
 // are read after waiting for the previous kernel on the stream; with the
@@ -33,6 +33,11 @@ namespace bsr {
 // activation rows, 8 for more (their per-row register arrays grow).
 template <int MR>
 constexpr int decode_max_warps() { return MR <= 2 ? 32 : 8; }
+
+// 1 KB chunks per bulk copy of a weight row: a weight-sized stream of
+// 1 KB copies measured at well under half the HBM rate of 16 KB copies
+// (each CTA issuing its share before the grid-dependency wait).
+constexpr uint32_t kChunksPerCopy = 16;
 
 __device__ __forceinline__ void bf16x8_to_f32_d(const uint4& v, float (&x)[8]) {
   x[0] = __uint_as_float(v.x << 16);
@@ -142,20 +147,25 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
     fence_mbar_init();
   }
   __syncwarp();
-  // A row goes out as 1 KB chunks (one 32-block per lane), each completing
-  // on its own barrier, so the first chunks can be consumed while the rest
-  // of the weight is still streaming.
+  // A row goes out as bulk copies of up to kChunksPerCopy 1 KB chunks (one
+  // 32-block per lane per chunk); a row longer than one copy is consumed
+  // copy by copy while its tail still streams.
   auto issue_row = [&](int r) {
     if (lane == 0 && r < n) {
       const int8_t* wr;
       const float* wsr;
       seg_row(r, wr, wsr);
-      for (uint32_t c = 0; c < L.chunks; ++c) {
-        const uint32_t blocks = min(32u, (uint32_t)nb - 32u * c);
+      // up to kChunksPerCopy chunks (and their scales) per bulk copy, on the
+      // group's first barrier; the group's other barriers complete at once,
+      // so the consumer's per-chunk waits are unchanged
+      for (uint32_t c0 = 0; c0 < L.chunks; c0 += kChunksPerCopy) {
+        const uint32_t cn = min(kChunksPerCopy, L.chunks - c0);
+        const uint32_t blocks = min(32u * cn, (uint32_t)nb - 32u * c0);
         const uint32_t wb = blocks * 32u, sb = L.wscale_bytes ? blocks * 4u : 0u;
-        mbar_arrive_expect_tx(&bars[c], wb + sb);
-        bulk_load(s_w + (size_t)c * 1024, wr + (size_t)c * 1024, wb, &bars[c]);
-        if (sb) bulk_load(s_ws + (size_t)c * 32, wsr + (size_t)c * 32, sb, &bars[c]);
+        mbar_arrive_expect_tx(&bars[c0], wb + sb);
+        bulk_load(s_w + (size_t)c0 * 1024, wr + (size_t)c0 * 1024, wb, &bars[c0]);
+        if (sb) bulk_load(s_ws + (size_t)c0 * 32, wsr + (size_t)c0 * 32, sb, &bars[c0]);
+        for (uint32_t c = c0 + 1; c < c0 + cn; ++c) mbar_arrive(&bars[c]);
       }
     }
   };

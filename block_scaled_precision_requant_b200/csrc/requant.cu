@@ -8,10 +8,8 @@
 //    elements (gemm_dense_int8.rs, `requant_a_kernel` inside
 //    `int8_gemm_faith2_prefill`).  The scales are written block-major,
 //    a_scale_t[K/32][ld], which is the layout the tensor-core GEMM stages.
-#include <cuda_fp16.h>
-#include <cuda_fp8.h>
-
 #include "common.cuh"
+#include "fp_cvt.cuh"
 #include "kernels.h"
 #include "quant.cuh"
 
@@ -28,12 +26,6 @@ namespace bsr {
 // nibble to its code with byte permutes; codes of negative nibbles are the
 // negated codes (rint half-even and the division are odd functions).
 // ---------------------------------------------------------------------------
-
-__device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
-  // hardware conversion E4M3 -> f16 (exact), then f16 -> f32 (exact)
-  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3);
-  return __half2float(__half(h));
-}
 
 // E2M1 magnitude of index i (0..7): 0, .5, 1, 1.5, 2, 3, 4, 6.
 __device__ __forceinline__ float e2m1_mag(uint32_t i) {
@@ -115,9 +107,10 @@ __global__ void __launch_bounds__(256) requant_w_kernel(const uint4* __restrict_
   for (long long gi = (long long)blockIdx.x * blockDim.x + threadIdx.x; gi < groups;
        gi += (long long)gridDim.x * blockDim.x) {
     const uint4 p = __ldg(w_packed + gi);
-    const uint32_t e = __ldg(w_e4m3 + gi);
-    const float s0 = e4m3_to_f32(e & 0xFFu);
-    const float s1 = e4m3_to_f32(e >> 8);
+    // both E4M3 scales of the group by one hardware conversion (exact)
+    const uint32_t e2 = e4m3x2_to_f16x2(__ldg(w_e4m3 + gi));
+    const float s0 = f16_lo_to_f32(e2);
+    const float s1 = f16_hi_to_f32(e2);
     const uint32_t i0 = max_mag_index(p.x, p.y);
     const uint32_t i1 = max_mag_index(p.z, p.w);
     const float a0 = fabsf(__fmul_rn(e2m1_mag(i0) * s0, scale2));

@@ -125,6 +125,9 @@ def test_source_hash_follows_the_kernels_own_sources(tmp_path, monkeypatch):
     csrc = _csrc_copy(tmp_path, monkeypatch)
     assert bench.kernel_sources("decode_kernel") == ["api.cu", "common.cuh", "decode.cu", "kernels.h", "quant.cuh"]
     assert bench.kernel_sources("gemm_kernel") == ["api.cu", "common.cuh", "gemm_tc.cu", "kernels.h"]
+    # a kernel launched from two layers depends on both
+    assert bench.kernel_sources("nvfp4_gemv_kernel") == ["api.cu", "common.cuh", "fp_cvt.cuh", "kernels.h",
+                                                         "nvfp4_enc.cuh", "nvfp4_gemv.cu", "w4a4.cu"]
     h = {k: bench.kernel_source_hash(k) for k in bench.KERNEL_UNITS}
     # a new, unrelated translation unit changes neither
     (csrc / "other.cu").write_text("__global__ void other_kernel() {}\n")
