@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbsr.so")
 SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "nvfp4_gemv.cu",
            "w4a4.cu", "w4a4_gemm.cu"]
-HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh", "w4a4_desc.cuh", "fp_cvt.cuh"]
+HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh", "w4a4_desc.cuh", "fp_cvt.cuh", "occupancy.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -199,11 +199,15 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1)
   };
 
   if (threadIdx.x == 0) *abort_flag = 0;
+  if (A4 && threadIdx.x < MR) s_amax[threadIdx.x] = 0.0f;  // row maxima of the one-pass quantiser
   if (bulk && lane == 0) {
     for (int s = 0; s < slots; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
-  __syncwarp();
+  if (A4)
+    __syncthreads();
+  else
+    __syncwarp();
   const int first = min(slots, my_st);
   // Launched with programmatic stream serialisation: wait for the previous
   // kernel on the stream before reading what it may have written (the
@@ -216,44 +220,17 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1)
     for (int j = 0; j < first; ++j) issue(j);
 
   // ---- the CTA's activation rows into shared memory ----
-  if constexpr (A4) {
-    // row scale2 from the row's largest magnitude
-#pragma unroll
-    for (int r = 0; r < MR; ++r) {
-      float mx = 0.0f;
-      if (r < rows) {
-        const uint4* src = reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * (size_t)k);
-        for (int i = threadIdx.x; i < nb; i += blockDim.x)
-          mx = fmaxf(mx, bf16x16_amax_f32(__ldg(src + 2 * i), __ldg(src + 2 * i + 1)));
-      }
-#pragma unroll
-      for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
-      if (lane == 0) s_amax[r * nwarps + warp] = mx;
-    }
-    __syncthreads();
-    if (threadIdx.x < MR) {
-      const int r = threadIdx.x;
-      float mx = 0.0f;
-      for (int w = 0; w < nwarps; ++w) mx = fmaxf(mx, s_amax[r * nwarps + w]);
-      s_s2[r] = r < rows ? nvfp4::row_scale2(mx) : 0.0f;
-    }
-    __syncthreads();
-  }
-  for (int i = threadIdx.x; i < MR * nb; i += blockDim.x) {
+  // one 16-block: W4A16 scaled f16 and 2^-s, W4A4 the E2M1 values of its
+  // NVFP4 codes (row scale s2) and its E4M3 scale
+  auto store_block = [&](int i, const uint4& v0, const uint4& v1, float s2) {
     const int r = i / nb;
     const int b = i - r * nb;
-    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
-    if (r < rows) {
-      const uint4* src = reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * (size_t)k + (size_t)b * 16);
-      v0 = __ldg(src);
-      v1 = __ldg(src + 1);
-    }
     uint4 h0, h1;
     float f;
     if constexpr (A4) {
       float x[16];
       bf16x16_to_f32(v0, v1, x);
-      const nvfp4::Block q = nvfp4::quant_block(x, s_s2[r]);
+      const nvfp4::Block q = nvfp4::quant_block(x, s2);
       uint32_t w[8];
       e2m1x8_to_f16x2(q.lo, &w[0]);
       e2m1x8_to_f16x2(q.hi, &w[4]);
@@ -261,12 +238,75 @@ __global__ void __launch_bounds__(kGemvMaxWarps * 32, 1)
       h1 = make_uint4(w[4], w[5], w[6], w[7]);
       f = e4m3_to_f32_hw(q.e4);
     } else {
+      (void)s2;
       f = a16_block(v0, v1, h0, h1);
     }
     uint8_t* row_act = smem + L.act + (size_t)r * (size_t)k * 2;
     *reinterpret_cast<uint4*>(row_act + act_half((uint32_t)b, 0)) = h0;
     *reinterpret_cast<uint4*>(row_act + act_half((uint32_t)b, 1)) = h1;
     s_fac[i] = f;
+  };
+  auto load_block = [&](int i, uint4& v0, uint4& v1) {
+    const int r = i / nb;
+    const int b = i - r * nb;
+    v0 = make_uint4(0, 0, 0, 0);
+    v1 = make_uint4(0, 0, 0, 0);
+    if (r < rows) {
+      const uint4* src = reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * (size_t)k + (size_t)b * 16);
+      v0 = __ldg(src);
+      v1 = __ldg(src + 1);
+    }
+  };
+  if constexpr (A4) {
+    if (MR * nb <= (int)blockDim.x) {
+      // one block per thread, kept in registers across the row reduction
+      // (row maxima by atomic max on the float bits, which order as
+      // unsigned integers for non-negative values)
+      const int i = threadIdx.x;
+      const bool mine = i < MR * nb;
+      uint4 v0 = make_uint4(0, 0, 0, 0), v1 = make_uint4(0, 0, 0, 0);
+      if (mine) {
+        load_block(i, v0, v1);
+        const uint32_t bits = bf16x16_absmax_bits(v0, v1) << 16;
+        if (bits) atomicMax(reinterpret_cast<unsigned int*>(s_amax) + i / nb, bits);
+      }
+      __syncthreads();
+      if (threadIdx.x < MR) s_s2[threadIdx.x] = (int)threadIdx.x < rows ? nvfp4::row_scale2(s_amax[threadIdx.x]) : 0.0f;
+      if (mine) store_block(i, v0, v1, i / nb < rows ? nvfp4::row_scale2(s_amax[i / nb]) : 0.0f);
+    } else {
+      // row maxima first (all threads), then the blocks
+#pragma unroll
+      for (int r = 0; r < MR; ++r) {
+        float mx = 0.0f;
+        if (r < rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(a + (size_t)(m0 + r) * (size_t)k);
+          for (int i = threadIdx.x; i < nb; i += blockDim.x)
+            mx = fmaxf(mx, bf16x16_amax_f32(__ldg(src + 2 * i), __ldg(src + 2 * i + 1)));
+        }
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+        if (lane == 0) s_amax[r * nwarps + warp] = mx;
+      }
+      __syncthreads();
+      if (threadIdx.x < MR) {
+        const int r = threadIdx.x;
+        float mx = 0.0f;
+        for (int w = 0; w < nwarps; ++w) mx = fmaxf(mx, s_amax[r * nwarps + w]);
+        s_s2[r] = r < rows ? nvfp4::row_scale2(mx) : 0.0f;
+      }
+      __syncthreads();
+      for (int i = threadIdx.x; i < MR * nb; i += blockDim.x) {
+        uint4 v0, v1;
+        load_block(i, v0, v1);
+        store_block(i, v0, v1, s_s2[i / nb]);
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < MR * nb; i += blockDim.x) {
+      uint4 v0, v1;
+      load_block(i, v0, v1);
+      store_block(i, v0, v1, 0.0f);
+    }
   }
   __syncthreads();
 

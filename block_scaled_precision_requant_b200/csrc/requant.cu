@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "fp_cvt.cuh"
 #include "kernels.h"
+#include "occupancy.h"
 #include "quant.cuh"
 
 namespace bsr {
@@ -204,7 +205,7 @@ static int grid_for(long long work_items, int per_block, int max_blocks) {
 cudaError_t launch_requant_w(const uint8_t* w_packed, const uint8_t* w_e4m3, float scale2, int8_t* w_i8,
                              float* w_scale, long long n, long long k, cudaStream_t stream, int num_sms) {
   const long long groups = n * (k / 32);
-  const int grid = grid_for(groups, 256, num_sms * 8);
+  const int grid = grid_for(groups, 256, num_sms * resident_ctas_per_sm((const void*)requant_w_kernel, 256));
   requant_w_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(w_packed),
                                              reinterpret_cast<const uint16_t*>(w_e4m3), scale2,
                                              reinterpret_cast<uint4*>(w_i8), w_scale, groups);
@@ -215,7 +216,7 @@ cudaError_t launch_requant_a(const uint16_t* a, int8_t* a_i8, float* a_scale_t, 
                              cudaStream_t stream, int num_sms) {
   // warp tasks of 8 rows x 4 blocks, 8 warps per CTA
   const long long tasks = (long long)((m + 7) / 8) * ((k / 32 + 3) / 4);
-  const int grid = grid_for(tasks, 8, num_sms * 8);
+  const int grid = grid_for(tasks, 8, num_sms * resident_ctas_per_sm((const void*)requant_a_kernel, 256));
   requant_a_kernel<<<grid, 256, 0, stream>>>(a, a_i8, a_scale_t, m, k, ld);
   return cudaGetLastError();
 }

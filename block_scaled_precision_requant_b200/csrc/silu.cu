@@ -28,6 +28,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "occupancy.h"
 #include "quant.cuh"
 
 namespace bsr {
@@ -148,7 +149,7 @@ int grid_for(long long work_items, int per_block, int max_blocks) {
 cudaError_t launch_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* x, int m, int k, cudaStream_t stream,
                             int num_sms) {
   const long long n8 = (long long)m * k / 8;
-  const int grid = grid_for(n8, 256, num_sms * 8);
+  const int grid = grid_for(n8, 256, num_sms * resident_ctas_per_sm((const void*)silu_mul_kernel, 256));
   silu_mul_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<const uint4*>(g), reinterpret_cast<const uint4*>(u),
                                             reinterpret_cast<uint4*>(x), n8);
   return cudaGetLastError();
@@ -157,7 +158,7 @@ cudaError_t launch_silu_mul(const uint16_t* g, const uint16_t* u, uint16_t* x, i
 cudaError_t launch_requant_silu_a(const uint16_t* g, const uint16_t* u, int8_t* a_i8, float* a_scale_t, int m, int k,
                                   int ld, cudaStream_t stream, int num_sms) {
   const long long tasks = (long long)((m + 7) / 8) * ((k / 32 + 3) / 4);
-  const int grid = grid_for(tasks, 8, num_sms * 8);
+  const int grid = grid_for(tasks, 8, num_sms * resident_ctas_per_sm((const void*)requant_silu_a_kernel, 256));
   requant_silu_a_kernel<<<grid, 256, 0, stream>>>(g, u, a_i8, a_scale_t, m, k, ld);
   return cudaGetLastError();
 }
