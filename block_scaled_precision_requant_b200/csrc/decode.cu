@@ -190,13 +190,19 @@ __global__ void __launch_bounds__(decode_max_warps<MR>() * 32, 1)
     // that kernel to complete (and its writes to be visible) before reading
     // what it may have written, and let the next kernel be scheduled early in
     // turn.  With static_weight the caller guarantees that no kernel ahead
-    // on the stream writes the weight, so the first row's copies go out
-    // before the wait and overlap the previous kernel's tail.
-    if (static_weight) issue_row(row);
+    // on the stream writes the weight, so the first eighth of the warps (at
+    // least one) send their first row's copies before the wait, overlapping
+    // the previous kernel's tail; the rest send theirs once the activation
+    // loads are out.  Issuing every warp's row before the wait queues the
+    // activation loads behind the whole first wave of the weight stream and
+    // delays the requantisation that every row needs (slower at M=1,
+    // N=K=4096 by about 15%); issuing none leaves the tail unused.
+    const bool early = static_weight && warp < (nwarps + 7) / 8;
+    if (early) issue_row(row);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     uint4 av = load_act(warp * 8);
-    if (!static_weight) issue_row(row);
+    if (!early) issue_row(row);
     for (int g0 = warp * 8; g0 < groups; g0 += nwarps * 8) {
       const int g = g0 + (lane >> 2);
       const int r = g / nb;

@@ -179,8 +179,8 @@ bsr_status bsr_gemm_partials(const int8_t* a_i8, const float* a_scale_t, const i
 
 /* bsr_decode_ex flag: no kernel that writes w_i8 or w_scale is in flight or
  * queued ahead of this call on the stream (e.g. a decode loop over a
- * resident weight).  The kernel then issues its first weight copies before
- * waiting for the previous kernel on the stream, so they overlap that
+ * resident weight).  The kernel then issues part of its first weight copies
+ * before waiting for the previous kernel on the stream, so they overlap that
  * kernel's tail.  Activations are still read only after that wait. */
 #define BSR_DECODE_STATIC_WEIGHT 1u
 
