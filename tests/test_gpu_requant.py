@@ -84,6 +84,14 @@ def test_requant_a_edge_rows(m):
     _check_a(a)
 
 
+@pytest.mark.parametrize("m,k", [(37, 2080), (9, 1024), (130, 3168), (8, 32)])
+def test_requant_a_ragged_column_tiles(m, k):
+    """K spanning several 1024-column tiles with a ragged last tile, and
+    row counts around the 8-row tile."""
+    a, _ = synth.make_activations(m, k, seed=k + m, recipe="laplace_zero_row")
+    _check_a(a)
+
+
 def test_requant_a_specials():
     # zero groups, subnormal BF16, huge values, exact halves (ties)
     k = 128
