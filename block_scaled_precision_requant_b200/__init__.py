@@ -347,8 +347,8 @@ def decode(a, w_i8, w_scale, out=None, stream=None, static_weight=False):
 
     ``static_weight=True`` promises that no kernel in flight or queued ahead
     on the stream writes ``w_i8``/``w_scale`` (a decode loop over a resident
-    weight); the kernel then starts its weight copies before waiting for the
-    previous kernel."""
+    weight); the kernel then starts part of its weight copies before waiting
+    for the previous kernel."""
     torch = _torch()
     m, k = a.shape
     n = w_i8.shape[0]

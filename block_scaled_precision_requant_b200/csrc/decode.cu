@@ -17,7 +17,8 @@
 // into shared memory (same rule and code as requant_a, so the codes match it
 // bit for bit).  Launched with programmatic dependent launch: activations
 // are read after waiting for the previous kernel on the stream; with the
-// static-weight option the first row's copies go out before that wait.  The
+// static-weight option an eighth of the warps send their first row's copies
+// before that wait.  The
 // weight is one [N, K] tensor or a table of stacked segments.
 #include <cuda_bf16.h>
 

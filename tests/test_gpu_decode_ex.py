@@ -1,5 +1,5 @@
 """bsr_decode_ex: the static-weight option only reorders the kernel's copies
-(weight copies issued before the wait on the previous kernel), so outputs
+(part of the weight copies issued before the wait on the previous kernel), so outputs
 must be bit-identical to bsr_decode and within tolerance of the oracle; also
 run as a CUDA-graph loop over two weight copies as the benchmark does."""
 import numpy as np
