@@ -19,8 +19,10 @@ copy of the requantised weight (copies cover >= 3x L2), timed with CUDA events
 around the replay.  Prefill: L2 is flushed (a 256 MiB device write) before
 every timed step, outside the per-step CUDA events.  ``ms_per_step`` is the
 mean step time.
-``e2e`` repeats the step through the public API with the activations copied
-in from pinned host memory and the output copied back inside the events.
+``e2e`` repeats the step through the public API with the activations moved
+in from pinned host memory and the output moved back inside the events: for
+decode through ``bsr_decode_host`` (copy kernels chained with the decode
+kernel), for prefill by stream copies around ``bsr_proj``.
 Under torchrun every rank runs the same workload on its own GPU (independent
 replicas: the path has no exchange step), timings are max-reduced over ranks.
 ``--impl reference`` times the CPU oracle (oracle/) on the host cores on a
@@ -401,6 +403,10 @@ class Gpu:
         self.bsr.proj(self.a, self.w_i8, self.w_s, self.out, self.scratch if self.scratch.numel() > 1 else None)
 
     def step_e2e(self):
+        m = self.wl.shape[0]
+        if m <= self.bsr.DECODE_MAX_M:
+            self.bsr.decode_host(self.a_host, self.w_i8, self.w_s, self.out_host, self.a, self.out)
+            return
         self.a.copy_(self.a_host, non_blocking=True)
         self.step()
         self.out_host.copy_(self.out, non_blocking=True)
@@ -450,10 +456,12 @@ class Gpu:
 
     def timed_e2e_graph(self, steps, warmup):
         """End to end through the public API as a decode loop runs it: every
-        step copies its activations from pinned host memory, runs the
-        projection, and copies the result back to pinned host memory; the K
-        steps are captured in one CUDA graph (so the host's Python overhead
-        is not what is measured) over rotating weight copies (>= 3x L2)."""
+        step reads its activations from pinned host memory, runs the decode
+        kernel and writes the result back to pinned host memory
+        (``bsr_decode_host``: copy kernels chained with the decode kernel);
+        the K steps are captured in one CUDA graph (so the host's Python
+        overhead is not what is measured) over rotating weight copies
+        (>= 3x L2)."""
         torch, bsr = self.torch, self.bsr
         l2 = torch.cuda.get_device_properties(self.dev).L2_cache_size
         wbytes = self.w_i8.numel() + 4 * self.w_s.numel()
@@ -461,10 +469,8 @@ class Gpu:
         ws = [(self.w_i8.clone(), self.w_s.clone()) for _ in range(copies)]
 
         def one(i):
-            self.a.copy_(self.a_host, non_blocking=True)
             w, s = ws[i % copies]
-            bsr.decode(self.a, w, s, self.out, static_weight=True)
-            self.out_host.copy_(self.out, non_blocking=True)
+            bsr.decode_host(self.a_host, w, s, self.out_host, self.a, self.out, static_weight=True)
 
         for i in range(max(warmup, 1)):
             one(i)
@@ -1138,8 +1144,9 @@ def gpu_main(args):
         "config": {**workload_desc(wl, world), "inputs_sha256": input_hashes(g.host)},
         "roofline": rl,
         "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": 2 * m * k, "d2h_bytes_per_step": 2 * m * n,
-                "how": ("CUDA graph of the K steps (copy in, projection, copy out each step)" if decode else
-                        "eager calls per step (copy in, projection, copy out)"),
+                "how": ("CUDA graph of the K steps through bsr_decode_host (copy kernel in, decode, copy "
+                        "kernel out each step)" if decode else
+                        "eager calls per step (stream copy in, projection, stream copy out)"),
                 "eager_value": world * units / (ms_e2e_eager / 1e3),
                 "ms_per_step": ms_e2e},
         "gpu_launches": g.launches_per_step() * args.steps,

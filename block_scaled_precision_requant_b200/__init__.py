@@ -101,6 +101,7 @@ SIGNATURES = [
     ("bsr_proj_noalloc", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     ("bsr_debug_wait_timeout", ctypes.c_int, [ctypes.c_int, _P]),
     ("bsr_decode_ex", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
+    ("bsr_decode_host", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_uint, _P]),
     ("bsr_decode_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_proj_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_w4a16_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
@@ -191,6 +192,23 @@ def _dev(t, dtype, shape, name):
         raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _host(t, dtype, shape, name):
+    """A page-locked host tensor (its address; the library checks that it is
+    mapped into the device's address space)."""
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must have dtype {dtype}, got {t.dtype}")
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     if not t.is_contiguous():
@@ -368,6 +386,33 @@ def decode(a, w_i8, w_scale, out=None, stream=None, static_weight=False):
         )
     )
     return out
+
+
+def decode_host(a_host, w_i8, w_scale, out_host, a_dev, out_dev, stream=None, static_weight=False):
+    """The decode step with the activations read from, and the result written
+    to, page-locked host tensors (``tensor.pin_memory()``); ``a_dev`` [M, K]
+    and ``out_dev`` [M, N] BF16 are device staging buffers.  The copies are
+    kernels chained with the decode kernel by programmatic dependent launch.
+    ``out_host`` holds the result once the stream has passed the call."""
+    torch = _torch()
+    m, k = a_host.shape
+    n = w_i8.shape[0]
+    _check(
+        lib().bsr_decode_host(
+            _host(a_host, torch.bfloat16, (m, k), "a_host"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _host(out_host, torch.bfloat16, (m, n), "out_host"),
+            m,
+            n,
+            k,
+            _dev(a_dev, torch.bfloat16, (m, k), "a_dev"),
+            _dev(out_dev, torch.bfloat16, (m, n), "out_dev"),
+            DECODE_STATIC_WEIGHT if static_weight else 0,
+            _stream_ptr(stream),
+        )
+    )
+    return out_host
 
 
 def debug_wait_timeout(limit_ms: int, stream=None):

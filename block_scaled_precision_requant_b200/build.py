@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbsr.so")
 SOURCES = ["api.cu", "requant.cu", "decode.cu", "gemm_tc.cu", "noalloc.cu", "debug.cu", "silu.cu", "nvfp4_gemv.cu",
-           "w4a4.cu", "w4a4_gemm.cu"]
+           "w4a4.cu", "w4a4_gemm.cu", "host_io.cu"]
 HEADERS = ["common.cuh", "quant.cuh", "kernels.h", "nvfp4_enc.cuh", "w4a4_desc.cuh", "fp_cvt.cuh", "occupancy.h"]
 
 NVCC_FLAGS = [

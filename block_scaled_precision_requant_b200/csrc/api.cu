@@ -399,6 +399,54 @@ bsr_status bsr_decode_ex(const uint16_t* a, const int8_t* w_i8, const float* w_s
   return decode_impl(a, w_i8, w_scale, out, m, n, k, stream, (flags & BSR_DECODE_STATIC_WEIGHT) ? 1 : 0);
 }
 
+// The device address of a page-locked host buffer mapped into the current
+// device's address space; nullptr when `p` is not one.
+static const void* mapped_host(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
+  return at.devicePointer;
+}
+
+bsr_status bsr_decode_host(const uint16_t* a_host, const int8_t* w_i8, const float* w_scale, uint16_t* out_host,
+                           int64_t m, int64_t n, int64_t k, uint16_t* a_dev, uint16_t* out_dev, unsigned flags,
+                           void* stream) {
+  if (flags & ~(unsigned)BSR_DECODE_STATIC_WEIGHT)
+    return fail(BSR_EINVAL, "bsr_decode_host: unknown flags 0x%x", flags);
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (m == 0 || n == 0) return ok();
+  if (!a_host || !out_host) return fail(BSR_EINVAL, "null pointer");
+  if ((st = check_proj_args(a_dev, w_i8, w_scale, out_dev)) != BSR_OK) return st;
+  if (!aligned16(a_host) || !aligned16(out_host) || !aligned16(out_dev))
+    return fail(BSR_EALIGN, "bsr_decode_host: a_host, out_host, a_dev, out_dev must be 16-byte aligned");
+  DevInfo d;
+  int mr = 0;
+  if ((st = decode_mr(m, k, d, mr)) != BSR_OK) return st;
+  const void* a_map = mapped_host(a_host);
+  void* out_map = const_cast<void*>(mapped_host(out_host));
+  if (!a_map || !out_map)
+    return fail(BSR_EINVAL, "bsr_decode_host: a_host and out_host must be page-locked host memory mapped into "
+                            "the device's address space");
+  // the decode launch's configuration before anything is queued
+  if ((st = cuda_status(bsr::prepare_decode((int)n, (int)k, mr, d.smem_optin, d.num_sms), "decode setup")) != BSR_OK)
+    return st;
+  cudaStream_t cs = as_stream(stream);
+  if ((st = cuda_status(bsr::launch_host_copy(a_map, a_dev, (size_t)m * (size_t)k * 2, cs, d.num_sms),
+                        "input copy launch")) != BSR_OK)
+    return st;
+  if ((st = cuda_status(bsr::launch_decode(a_dev, w_i8, w_scale, out_dev, (int)m, (int)n, (int)k, mr,
+                                           (flags & BSR_DECODE_STATIC_WEIGHT) ? 1 : 0, d.status, d.smem_optin, cs,
+                                           d.num_sms),
+                        "decode launch")) != BSR_OK)
+    return st;
+  return cuda_status(bsr::launch_host_copy(out_dev, out_map, (size_t)m * (size_t)n * 2, cs, d.num_sms),
+                     "output copy launch");
+}
+
 bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m, int64_t n,
                     int64_t k, void* scratch, size_t scratch_bytes, void* stream) {
   bsr_status st = check_dims(m, n, k, true, true);

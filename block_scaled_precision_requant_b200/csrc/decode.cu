@@ -309,35 +309,44 @@ int decode_rows_per_cta(int m, int k, size_t smem_limit) {
   return fits(mr) ? mr : 0;
 }
 
+// Warps per CTA and dynamic shared memory of a launch over n weight rows,
+// with the kernel's shared-memory opt-in (raised once per device and
+// variant, under a lock shared by all variants).
+template <int MR, class Src>
+static cudaError_t decode_config(int n, int k, size_t smem_limit, int num_sms, int& w, size_t& smem) {
+  const bool sb = decode_scale_bulk(k);
+  // Warps (= weight rows in flight) per CTA: spread the rows over all SMs,
+  // at most decode_max_warps<MR>() per CTA and as many row slots as fit in
+  // shared memory; beyond one CTA per SM the warps loop over rows.
+  constexpr int kMaxW = decode_max_warps<MR>();
+  w = (int)((n + (long long)num_sms - 1) / num_sms);
+  w = w < 1 ? 1 : (w > kMaxW ? kMaxW : w);
+  while (w > 1 && decode_smem_layout(MR, k, w, sb).total > smem_limit) --w;
+  smem = decode_smem_layout(MR, k, w, sb).total;
+  static size_t granted[64] = {};  // per device, per <MR, Src>
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_decode_optin_mu);
+  if (smem > granted[dev]) {
+    e = cudaFuncSetAttribute(decode_kernel<MR, Src>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    granted[dev] = smem;
+  }
+  return cudaSuccess;
+}
+
 template <int MR, class Src>
 static cudaError_t launch_decode_t(const uint16_t* a, const Src& src, int n, uint16_t* out, int m, int k,
                                    int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
                                    int num_sms) {
   auto kern = decode_kernel<MR, Src>;
   const bool sb = decode_scale_bulk(k);
-  // Warps (= weight rows in flight) per CTA: spread the rows over all SMs,
-  // at most decode_max_warps<MR>() per CTA and as many row slots as fit in
-  // shared memory; beyond one CTA per SM the warps loop over rows.
-  constexpr int kMaxW = decode_max_warps<MR>();
-  int w = (int)((n + (long long)num_sms - 1) / num_sms);
-  w = w < 1 ? 1 : (w > kMaxW ? kMaxW : w);
-  while (w > 1 && decode_smem_layout(MR, k, w, sb).total > smem_limit) --w;
-  const size_t smem = decode_smem_layout(MR, k, w, sb).total;
-  // dynamic shared-memory limit granted so far, per device (per <MR, Src>),
-  // raised under a lock shared by all variants
-  static size_t granted[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  int w = 1;
+  size_t smem = 0;
+  cudaError_t e = decode_config<MR, Src>(n, k, smem_limit, num_sms, w, smem);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  {
-    std::lock_guard<std::mutex> lk(g_decode_optin_mu);
-    if (smem > granted[dev]) {
-      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-      granted[dev] = smem;
-    }
-  }
   const int gy = (m + MR - 1) / MR;
   long long gx = (n + w - 1) / w;
   if (gx * gy > num_sms) gx = ((long long)num_sms + gy - 1) / gy;
@@ -367,6 +376,19 @@ static cudaError_t launch_decode_src(const uint16_t* a, const Src& src, int n, u
     case 4: return launch_decode_t<4, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
     case 8: return launch_decode_t<8, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
     case 16: return launch_decode_t<16, Src>(a, src, n, out, m, k, sw, status, smem_limit, stream, num_sms);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t prepare_decode(int n, int k, int mr, size_t smem_limit, int num_sms) {
+  int w = 1;
+  size_t smem = 0;
+  switch (mr) {
+    case 1: return decode_config<1, DecodeSingle>(n, k, smem_limit, num_sms, w, smem);
+    case 2: return decode_config<2, DecodeSingle>(n, k, smem_limit, num_sms, w, smem);
+    case 4: return decode_config<4, DecodeSingle>(n, k, smem_limit, num_sms, w, smem);
+    case 8: return decode_config<8, DecodeSingle>(n, k, smem_limit, num_sms, w, smem);
+    case 16: return decode_config<16, DecodeSingle>(n, k, smem_limit, num_sms, w, smem);
     default: return cudaErrorInvalidValue;
   }
 }

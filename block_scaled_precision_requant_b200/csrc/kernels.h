@@ -38,6 +38,13 @@ struct DecodeSegs {
 };
 
 int decode_rows_per_cta(int m, int k, size_t smem_limit);
+// The decode launch's configuration and shared-memory opt-in for a single
+// weight, made ahead of any launch (the launch itself repeats it, cached).
+cudaError_t prepare_decode(int n, int k, int mr, size_t smem_limit, int num_sms);
+// Copy of `bytes` (even) from src to dst by one or more CTAs, launched with
+// programmatic dependent launch; either side may be device-mapped host
+// memory.  Both pointers 16-byte aligned.
+cudaError_t launch_host_copy(const void* src, void* dst, size_t bytes, cudaStream_t stream, int num_sms);
 cudaError_t launch_decode(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int m, int n,
                           int k, int mr, int static_weight, int* status, size_t smem_limit, cudaStream_t stream,
                           int num_sms);

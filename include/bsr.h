@@ -190,6 +190,29 @@ bsr_status bsr_decode_ex(const uint16_t* a, const int8_t* w_i8, const float* w_s
                          int64_t n, int64_t k, unsigned flags, void* stream);
 
 /*
+ * Decode with the activations and the result in HOST memory: a decode loop
+ * driven by the host.  Same operation, results and errors as bsr_decode_ex
+ * (flags 0 or BSR_DECODE_STATIC_WEIGHT); out_host holds exactly the bits
+ * bsr_decode writes.
+ *   a_host   [M, K] BF16, page-locked host memory mapped into the device's
+ *            address space (cudaHostAlloc, or cudaHostRegister with the
+ *            mapped flag; with unified addressing every page-locked
+ *            allocation is), 16-byte aligned, owned by the caller;
+ *   out_host [M, N] BF16, the same kind of memory, 16-byte aligned;
+ *   a_dev    [M, K] BF16 and out_dev [M, N] BF16: device staging buffers
+ *            owned by the caller, 16-byte aligned.
+ * Three launches on `stream`, each with programmatic dependent launch: a
+ * copy kernel reads a_host into a_dev over the host link, the decode kernel
+ * computes out_dev, a copy kernel writes out_dev into out_host.  The host
+ * may read out_host (or rewrite a_host) only once the stream has passed
+ * this call.  A host buffer that is not page-locked and mapped gives
+ * BSR_EINVAL, with nothing launched.
+ */
+bsr_status bsr_decode_host(const uint16_t* a_host, const int8_t* w_i8, const float* w_scale, uint16_t* out_host,
+                           int64_t m, int64_t n, int64_t k, uint16_t* a_dev, uint16_t* out_dev, unsigned flags,
+                           void* stream);
+
+/*
  * Stacked weights (w8a8_decode/parts.rs, `W8a8Weight`: a weight stacked from
  * segments, e.g. Q, K and V, whose `segment(i)` "writes the bits the stacked
  * launch writes for those rows").  Segment s is a weight of its own

@@ -122,6 +122,19 @@ def test_nvfp4_gemv_ex_argument_errors(L):
     assert L.bsr_w4a16_decode_ex(_fake(264), _fake(256), _fake(256), f, _fake(256), 1, 8, 64, 1, None) == 2
 
 
+def test_decode_host_argument_errors(L):
+    ok = _fake(256)
+    assert L.bsr_decode_host(ok, ok, ok, ok, 1, 8, 64, ok, ok, 2, None) == 1
+    assert "flags" in bsr.last_error()
+    assert L.bsr_decode_host(None, None, None, None, 0, 8, 64, None, None, 0, None) == 0
+    assert L.bsr_decode_host(ok, ok, ok, ok, 1, 8, 48, ok, ok, 0, None) == 3
+    assert L.bsr_decode_host(None, ok, ok, ok, 1, 8, 64, ok, ok, 0, None) == 1
+    assert L.bsr_decode_host(ok, ok, ok, ok, 1, 8, 64, None, ok, 0, None) == 1
+    assert L.bsr_decode_host(_fake(264), ok, ok, ok, 1, 8, 64, ok, ok, 0, None) == 2
+    assert L.bsr_decode_host(ok, ok, ok, _fake(264), 1, 8, 64, ok, ok, 0, None) == 2
+    assert L.bsr_decode_host(ok, ok, ok, ok, 1, 8, 64, ok, _fake(258), 0, None) == 2
+
+
 def test_stacked_argument_errors(L):
     arr = (ctypes.c_void_p * 1)(_fake(256).value)
     n1 = (ctypes.c_int64 * 1)(8)
