@@ -102,6 +102,8 @@ SIGNATURES = [
     ("bsr_debug_wait_timeout", ctypes.c_int, [ctypes.c_int, _P]),
     ("bsr_decode_ex", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_decode_host", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, ctypes.c_uint, _P]),
+    ("bsr_proj_host_scratch_bytes", _I64, [_I64, _I64, _I64]),
+    ("bsr_proj_host", ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _P, ctypes.c_size_t, _I64, _P]),
     ("bsr_decode_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, ctypes.c_uint, _P]),
     ("bsr_proj_stacked", ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _P, ctypes.c_size_t, _P]),
     ("bsr_w4a16_decode", ctypes.c_int, [_P, _P, _P, ctypes.c_float, _P, _I64, _I64, _I64, _P]),
@@ -413,6 +415,44 @@ def decode_host(a_host, w_i8, w_scale, out_host, a_dev, out_dev, stream=None, st
         )
     )
     return out_host
+
+
+def proj_host(a_host, w_i8, w_scale, out_host, a_dev, out_dev, scratch=None, chunk_rows=0, stream=None):
+    """bsr_proj with page-locked host activations and result, pipelined over
+    row chunks (copies of one chunk overlap the compute of its neighbours).
+    ``a_dev`` [M, K] and ``out_dev`` [M, N] BF16 are device staging buffers;
+    ``scratch`` (uint8, device) of ``proj_host_scratch_bytes(M, K,
+    chunk_rows)`` bytes is allocated when not given."""
+    torch = _torch()
+    m, k = a_host.shape
+    n = w_i8.shape[0]
+    need = int(lib().bsr_proj_host_scratch_bytes(m, k, chunk_rows))
+    if scratch is None and need > 0:
+        scratch = torch.empty((need,), dtype=torch.uint8, device=a_dev.device)
+    ptr = ctypes.c_void_p(scratch.data_ptr()) if scratch is not None else None
+    size = scratch.numel() if scratch is not None else 0
+    _check(
+        lib().bsr_proj_host(
+            _host(a_host, torch.bfloat16, (m, k), "a_host"),
+            _dev(w_i8, torch.int8, (n, k), "w_i8"),
+            _dev(w_scale, torch.float32, (n, k // 32), "w_scale"),
+            _host(out_host, torch.bfloat16, (m, n), "out_host"),
+            m,
+            n,
+            k,
+            _dev(a_dev, torch.bfloat16, (m, k), "a_dev"),
+            _dev(out_dev, torch.bfloat16, (m, n), "out_dev"),
+            ptr,
+            size,
+            chunk_rows,
+            _stream_ptr(stream),
+        )
+    )
+    return out_host
+
+
+def proj_host_scratch_bytes(m: int, k: int, chunk_rows: int = 0) -> int:
+    return int(lib().bsr_proj_host_scratch_bytes(m, k, chunk_rows))
 
 
 def debug_wait_timeout(limit_ms: int, stream=None):

@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "bsr.h"
 #include "common.cuh"
@@ -447,6 +448,58 @@ bsr_status bsr_decode_host(const uint16_t* a_host, const int8_t* w_i8, const flo
                      "output copy launch");
 }
 
+// Copy streams and events of the host-buffer projection, created once per
+// device; the enqueue sequence that uses them runs under a lock.
+static constexpr int kMaxHostChunks = 64;
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t in[kMaxHostChunks] = {}, done[kMaxHostChunks] = {};
+};
+static HostPipe g_host_pipe[64];
+static std::mutex g_host_pipe_mu;
+
+static bsr_status host_pipe(int dev, HostPipe*& out) {
+  if (dev < 0 || dev >= 64) return fail(BSR_ENODEV, "device index %d out of range", dev);
+  HostPipe& hp = g_host_pipe[dev];
+  if (!hp.ready) {
+    cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.join, cudaEventDisableTiming);
+    for (int i = 0; e == cudaSuccess && i < kMaxHostChunks; ++i) {
+      e = cudaEventCreateWithFlags(&hp.in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done[i], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return fail(BSR_ECUDA, "host-buffer projection streams: %s", cudaGetErrorString(e));
+    hp.ready = true;
+  }
+  out = &hp;
+  return BSR_OK;
+}
+
+static bool is_pinned_host(const void* p) {
+  cudaPointerAttributes at;
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return false;
+  }
+  return at.type == cudaMemoryTypeHost;
+}
+
+static int64_t host_chunk_rows(int64_t m, int64_t chunk_rows) {
+  if (chunk_rows <= 0) {
+    // about four chunks, whole 128-row tiles, at least 512 rows
+    chunk_rows = (m + 3) / 4;
+    chunk_rows = (chunk_rows + 127) / 128 * 128;
+    if (chunk_rows < 512) chunk_rows = 512;
+  }
+  const int64_t min_rows = (m + kMaxHostChunks - 1) / kMaxHostChunks;
+  if (chunk_rows < min_rows) chunk_rows = min_rows;
+  return chunk_rows > m ? m : chunk_rows;
+}
+
 bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale, uint16_t* out, int64_t m, int64_t n,
                     int64_t k, void* scratch, size_t scratch_bytes, void* stream) {
   bsr_status st = check_dims(m, n, k, true, true);
@@ -468,6 +521,91 @@ bsr_status bsr_proj(const uint16_t* a, const int8_t* w_i8, const float* w_scale,
                         "requant_a launch")) != BSR_OK)
     return st;
   return gemm_run(p, out, nullptr, stream);
+}
+
+int64_t bsr_proj_host_scratch_bytes(int64_t m, int64_t k, int64_t chunk_rows) {
+  if (m <= 0 || k <= 0) return 0;
+  return (int64_t)bsr_proj_scratch_bytes(host_chunk_rows(m, chunk_rows), k);
+}
+
+bsr_status bsr_proj_host(const uint16_t* a_host, const int8_t* w_i8, const float* w_scale, uint16_t* out_host,
+                         int64_t m, int64_t n, int64_t k, uint16_t* a_dev, uint16_t* out_dev, void* scratch,
+                         size_t scratch_bytes, int64_t chunk_rows, void* stream) {
+  bsr_status st = check_dims(m, n, k, true, true);
+  if (st != BSR_OK) return st;
+  if (chunk_rows < 0) return fail(BSR_EINVAL, "bsr_proj_host: chunk_rows %lld < 0", (long long)chunk_rows);
+  if (m == 0 || n == 0) return ok();
+  if (!a_host || !out_host) return fail(BSR_EINVAL, "null pointer");
+  if ((st = check_proj_args(a_dev, w_i8, w_scale, out_dev)) != BSR_OK) return st;
+  const int64_t rows = host_chunk_rows(m, chunk_rows);
+  const int chunks = (int)((m + rows - 1) / rows);
+  const size_t need = bsr_proj_scratch_bytes(rows, k);
+  if (need && (!scratch || scratch_bytes < need))
+    return fail(BSR_ESCRATCH, "scratch of %zu bytes needed, %zu given", need, scratch ? scratch_bytes : (size_t)0);
+  if (need && (reinterpret_cast<uintptr_t>(scratch) & 255u) != 0)
+    return fail(BSR_EALIGN, "scratch must be 256-byte aligned");
+  if (!is_pinned_host(a_host) || !is_pinned_host(out_host))
+    return fail(BSR_EINVAL, "bsr_proj_host: a_host and out_host must be page-locked host memory");
+  DevInfo d;
+  if ((st = device_info(d)) != BSR_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(BSR_ENODEV, "cudaGetDevice failed");
+  // every chunk's launch prepared before anything is queued: the GEMM plan
+  // (tensor maps, opt-in) of a tensor-core chunk, the decode setup of a
+  // chunk the decode kernel serves (at most 16 rows, or K % 128 != 0)
+  std::vector<GemmPlan> plans((size_t)chunks);
+  std::vector<int> dec_mr((size_t)chunks, 0);
+  int8_t* a_i8 = static_cast<int8_t*>(scratch);
+  for (int c = 0; c < chunks; ++c) {
+    const int64_t r0 = (int64_t)c * rows, mc = (m - r0 < rows) ? m - r0 : rows;
+    if (mc <= BSR_DECODE_MAX_M || k % 128 != 0) {
+      DevInfo dd;
+      if ((st = decode_mr(mc, k, dd, dec_mr[c])) != BSR_OK) return st;
+      if ((st = cuda_status(bsr::prepare_decode((int)n, (int)k, dec_mr[c], dd.smem_optin, dd.num_sms),
+                            "decode setup")) != BSR_OK)
+        return st;
+    } else {
+      float* a_st = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)mc * (size_t)k));
+      if ((st = gemm_plan(plans[c], a_i8, a_st, w_i8, w_scale, out_dev + r0 * n, false, mc, n, k)) != BSR_OK)
+        return st;
+    }
+  }
+  std::lock_guard<std::mutex> lk(g_host_pipe_mu);
+  HostPipe* hp = nullptr;
+  if ((st = host_pipe(dev, hp)) != BSR_OK) return st;
+  cudaStream_t cs = as_stream(stream);
+  // the copy streams start after the work already queued on `stream`
+  if (cudaEventRecord(hp->fork, cs) != cudaSuccess || cudaStreamWaitEvent(hp->h2d, hp->fork, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->d2h, hp->fork, 0) != cudaSuccess)
+    return fail(BSR_ECUDA, "host-buffer projection fork failed");
+  for (int c = 0; c < chunks; ++c) {
+    const int64_t r0 = (int64_t)c * rows, mc = (m - r0 < rows) ? m - r0 : rows;
+    if (cudaMemcpyAsync(a_dev + r0 * k, a_host + r0 * k, (size_t)(mc * k) * 2, cudaMemcpyHostToDevice, hp->h2d) !=
+            cudaSuccess ||
+        cudaEventRecord(hp->in[c], hp->h2d) != cudaSuccess || cudaStreamWaitEvent(cs, hp->in[c], 0) != cudaSuccess)
+      return fail(BSR_ECUDA, "host-buffer projection: input copy of chunk %d failed", c);
+    if (dec_mr[c]) {
+      if ((st = cuda_status(bsr::launch_decode(a_dev + r0 * k, w_i8, w_scale, out_dev + r0 * n, (int)mc, (int)n,
+                                               (int)k, dec_mr[c], 0, d.status, d.smem_optin, cs, d.num_sms),
+                            "decode launch")) != BSR_OK)
+        return st;
+    } else {
+      float* a_st = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + align256((size_t)mc * (size_t)k));
+      if ((st = cuda_status(bsr::launch_requant_a(a_dev + r0 * k, a_i8, a_st, (int)mc, (int)k, (int)a_scale_ld(mc),
+                                                  cs, d.num_sms),
+                            "requant_a launch")) != BSR_OK ||
+          (st = gemm_run(plans[c], out_dev + r0 * n, nullptr, cs)) != BSR_OK)
+        return st;
+    }
+    if (cudaEventRecord(hp->done[c], cs) != cudaSuccess || cudaStreamWaitEvent(hp->d2h, hp->done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(out_host + r0 * n, out_dev + r0 * n, (size_t)(mc * n) * 2, cudaMemcpyDeviceToHost,
+                        hp->d2h) != cudaSuccess)
+      return fail(BSR_ECUDA, "host-buffer projection: output copy of chunk %d failed", c);
+  }
+  // `stream` passes this call once the last output copy has landed
+  if (cudaEventRecord(hp->join, hp->d2h) != cudaSuccess || cudaStreamWaitEvent(cs, hp->join, 0) != cudaSuccess)
+    return fail(BSR_ECUDA, "host-buffer projection join failed");
+  return ok();
 }
 
 bsr_status bsr_silu_mul(const uint16_t* gate, const uint16_t* up, uint16_t* x, int64_t m, int64_t k, void* stream) {

@@ -213,6 +213,30 @@ bsr_status bsr_decode_host(const uint16_t* a_host, const int8_t* w_i8, const flo
                            void* stream);
 
 /*
+ * bsr_proj with the activations and the result in HOST memory, pipelined:
+ * the rows go in chunks of `chunk_rows` (0: about four chunks of whole
+ * 128-row tiles, at least 512 rows; never more than 64 chunks), and while
+ * chunk c is requantised and multiplied on `stream`, chunk c+1 is copied in
+ * and chunk c-1 copied out on the library's own copy streams (DMA copies).
+ * Same operation, results and errors as bsr_proj on each chunk of rows: a
+ * row's bits do not depend on the other rows, so out_host holds exactly the
+ * bits bsr_proj writes.
+ *   a_host   [M, K] BF16 and out_host [M, N] BF16: page-locked host memory
+ *            (cudaHostAlloc / cudaHostRegister), owned by the caller;
+ *   a_dev    [M, K] BF16 (16-byte aligned) and out_dev [M, N] BF16: device
+ *            staging buffers owned by the caller;
+ *   scratch  bsr_proj_host_scratch_bytes(M, K, chunk_rows) bytes, 256-byte
+ *            aligned (0 bytes when every chunk takes the decode kernel).
+ * `stream` passes the call once the last chunk's result is in out_host. A
+ * host buffer that is not page-locked gives BSR_EINVAL, with nothing
+ * launched; every chunk's launch is prepared before the first is queued.
+ */
+int64_t bsr_proj_host_scratch_bytes(int64_t m, int64_t k, int64_t chunk_rows);
+bsr_status bsr_proj_host(const uint16_t* a_host, const int8_t* w_i8, const float* w_scale, uint16_t* out_host,
+                         int64_t m, int64_t n, int64_t k, uint16_t* a_dev, uint16_t* out_dev, void* scratch,
+                         size_t scratch_bytes, int64_t chunk_rows, void* stream);
+
+/*
  * Stacked weights (w8a8_decode/parts.rs, `W8a8Weight`: a weight stacked from
  * segments, e.g. Q, K and V, whose `segment(i)` "writes the bits the stacked
  * launch writes for those rows").  Segment s is a weight of its own

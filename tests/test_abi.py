@@ -135,6 +135,22 @@ def test_decode_host_argument_errors(L):
     assert L.bsr_decode_host(ok, ok, ok, ok, 1, 8, 64, ok, _fake(258), 0, None) == 2
 
 
+def test_proj_host_argument_errors(L):
+    ok = _fake(256)
+    # scratch sizes: one chunk's bsr_proj scratch; none for the decode route
+    assert L.bsr_proj_host_scratch_bytes(8192, 4096, 1024) == L.bsr_proj_scratch_bytes(1024, 4096)
+    assert L.bsr_proj_host_scratch_bytes(8192, 4096, 0) == L.bsr_proj_scratch_bytes(2048, 4096)
+    assert L.bsr_proj_host_scratch_bytes(16, 4096, 0) == 0
+    assert L.bsr_proj_host_scratch_bytes(100000, 4096, 8) == L.bsr_proj_scratch_bytes(1563, 4096)  # <= 64 chunks
+    args = (ok, ok, ok, ok, 4096, 64, 256, ok, ok)
+    assert L.bsr_proj_host(*args, ok, 1 << 30, -1, None) == 1
+    assert L.bsr_proj_host(None, None, None, None, 0, 64, 256, None, None, None, 0, 0, None) == 0
+    assert L.bsr_proj_host(ok, ok, ok, ok, 4096, 64, 48, ok, ok, ok, 1 << 30, 0, None) == 3
+    assert L.bsr_proj_host(None, ok, ok, ok, 4096, 64, 256, ok, ok, ok, 1 << 30, 0, None) == 1
+    assert L.bsr_proj_host(*args, None, 0, 0, None) == 4
+    assert L.bsr_proj_host(*args, _fake(272), 1 << 30, 0, None) == 2
+
+
 def test_stacked_argument_errors(L):
     arr = (ctypes.c_void_p * 1)(_fake(256).value)
     n1 = (ctypes.c_int64 * 1)(8)
