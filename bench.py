@@ -408,7 +408,9 @@ class Gpu:
         if m <= self.bsr.DECODE_MAX_M:
             self.bsr.decode_host(self.a_host, self.w_i8, self.w_s, self.out_host, self.a, self.out)
             return
-        self.bsr.proj_host(self.a_host, self.w_i8, self.w_s, self.out_host, self.a, self.out, self.scratch)
+        # 512-row chunks: the best of 256 / 512 / 1024 / 2048 / the default on
+        # the three prefill shapes together
+        self.bsr.proj_host(self.a_host, self.w_i8, self.w_s, self.out_host, self.a, self.out, self.scratch, 512)
 
     def launches_per_step(self):
         m, _, k = self.wl.shape
